@@ -1,0 +1,180 @@
+"""Seeded synthetic inputs for the NVFP4 W4A4 linear layer.
+
+This module is shared by the tests, the benchmark, the smoke check and the
+oracle-side checks.  It holds random-number plumbing only: it draws
+activations and weights with the shapes and statistics the pages describe,
+and contains none of the quantization or GEMM arithmetic.
+
+Statistics it imitates (no dataset is used, the pages' tensors are not
+available):
+  * activations share residual-stream outliers: median-layer max/RMS of about
+    63.5 and heavy tails (kurtosis in the thousands) [anthology record
+    LIT-800, "Key takeaways" (section 5.1, Table 2)];
+  * outlier channels reach 48-368x the RMS [LIT-800, "Standing in the
+    anthology"].
+Heavy tails come from a Student-t with 3 degrees of freedom; a fixed 0.1 %
+subset of channels (columns along K) is then scaled so the whole tensor's
+max/RMS lands on the target.
+
+Model dimensions (hidden 5120, MLP 17408, fused GDN in-projection segments
+8192/4096/48/48) are the workload definitions of this library's benchmark;
+the pages do not state them.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import torch
+
+# -------------------------------------------------------------------------
+# workloads
+# -------------------------------------------------------------------------
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    M: int
+    N: int
+    K: int
+    seed: int
+    x_kind: str           # "normal", "normal_outliers", "student_t"
+    x_dtype: str          # "float32" or "bfloat16"
+    segments: tuple = ()  # fused projection: rows of W per segment
+    seg_sigma: tuple = ()
+
+
+TINY = Workload("tiny", 16, 256, 256, 0, "normal", "float32")
+DECODE = Workload("decode", 8, 12288, 5120, 1, "normal_outliers", "bfloat16")
+PREFILL = Workload("prefill", 32768, 17408, 5120, 2, "student_t", "bfloat16")
+FUSED_GDN = Workload("fused_gdn", 4096, 12384, 5120, 3, "student_t", "bfloat16",
+                     segments=(8192, 4096, 48, 48),
+                     seg_sigma=(0.02, 0.02 / 4, 0.02 / 16, 0.02 / 64))
+QUANT_SWEEP_M = (1, 64, 4096, 32768)
+QUANT_SWEEP_K = (5120, 17408)
+QUANT_SWEEP_SEED = 4
+FUSED_SEGMENT_NAMES = ("qkv", "z", "a", "b")
+
+WORKLOADS = {w.name: w for w in (TINY, DECODE, PREFILL, FUSED_GDN)}
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def _dtype(name: str) -> torch.dtype:
+    return {"float32": torch.float32, "bfloat16": torch.bfloat16}[name]
+
+
+# -------------------------------------------------------------------------
+# activations
+# -------------------------------------------------------------------------
+
+
+def normal(shape, seed: int, std: float = 1.0, dtype=torch.float32, device="cpu"):
+    g = _gen(seed, device)
+    x = torch.randn(*shape, generator=g, device=device, dtype=torch.float32) * std
+    return x.to(dtype)
+
+
+def normal_with_outlier_channels(M: int, K: int, seed: int, factor: float = 60.0,
+                                 frac: float = 0.001, dtype=torch.bfloat16, device="cpu"):
+    """N(0,1) activations with a seeded 0.1 % channel subset multiplied by ``factor``."""
+    g = _gen(seed, device)
+    x = torch.randn(M, K, generator=g, device=device, dtype=torch.float32)
+    n_out = max(1, int(round(frac * K)))
+    idx = torch.randperm(K, generator=g, device=device)[:n_out]
+    x[:, idx] *= factor
+    return x.to(dtype)
+
+
+def student_t_outliers(M: int, K: int, seed: int, target_max_over_rms: float = 63.0,
+                       frac: float = 0.001, clip: float = 30.0, dtype=torch.bfloat16,
+                       device="cpu"):
+    """Heavy-tailed activations: Student-t(3) clipped at |t| <= clip, then a
+    seeded 0.1 % channel subset scaled so that max|x| / rms(x) is the target.
+
+    The scale factor f solves  f * m_c / sqrt((S_o + f^2 S_c)/n) = target  when
+    the outlier channels hold the maximum (m_c, S_c: their max and square sum;
+    S_o: the rest's square sum), which is a closed form in f^2.
+    """
+    g = _gen(seed, device)
+    z = torch.randn(M, K, generator=g, device=device, dtype=torch.float32)
+    chi = torch.zeros(M, K, device=device, dtype=torch.float32)
+    for _ in range(3):
+        e = torch.randn(M, K, generator=g, device=device, dtype=torch.float32)
+        chi.addcmul_(e, e)
+    t = z / torch.sqrt(chi / 3.0)
+    del chi, z
+    t.clamp_(-clip, clip)
+    n_out = max(1, int(round(frac * K)))
+    idx = torch.randperm(K, generator=g, device=device)[:n_out]
+    mask = torch.zeros(K, dtype=torch.bool, device=device)
+    mask[idx] = True
+    n = float(M) * K
+    s_c = float((t[:, mask].double() ** 2).sum())
+    s_o = float((t[:, ~mask].double() ** 2).sum())
+    m_c = float(t[:, mask].abs().max())
+    T2 = target_max_over_rms ** 2
+    # f^2 (m_c^2 - T2 s_c / n) = T2 s_o / n
+    denom = m_c * m_c - T2 * s_c / n
+    f = math.sqrt(T2 * s_o / n / denom) if denom > 0 else 1.0
+    f = max(f, 1.0)
+    t[:, mask] *= f
+    return t.to(dtype)
+
+
+def activation(w: Workload, device="cpu", M: int | None = None, K: int | None = None,
+               seed: int | None = None):
+    M = w.M if M is None else M
+    K = w.K if K is None else K
+    seed = w.seed if seed is None else seed
+    dt = _dtype(w.x_dtype)
+    if w.x_kind == "normal":
+        return normal((M, K), seed, 1.0, dt, device)
+    if w.x_kind == "normal_outliers":
+        return normal_with_outlier_channels(M, K, seed, dtype=dt, device=device)
+    if w.x_kind == "student_t":
+        return student_t_outliers(M, K, seed, dtype=dt, device=device)
+    raise ValueError(w.x_kind)
+
+
+def quant_sweep_activation(M: int, K: int, device="cpu"):
+    return student_t_outliers(M, K, QUANT_SWEEP_SEED + 1000 * M + K, dtype=torch.bfloat16,
+                              device=device)
+
+
+# -------------------------------------------------------------------------
+# weights
+# -------------------------------------------------------------------------
+
+
+def weight(w: Workload, device="cpu", N: int | None = None, K: int | None = None):
+    """W [N, K] ~ N(0, 0.02) (bf16 except the fp32 tiny case); for the fused
+    workload, the segments are drawn with their own standard deviations."""
+    N = w.N if N is None else N
+    K = w.K if K is None else K
+    dt = _dtype(w.x_dtype)
+    if not w.segments:
+        return normal((N, K), w.seed + 7919, 0.02, dt, device)
+    parts = []
+    for i, (rows, sd) in enumerate(zip(w.segments, w.seg_sigma)):
+        parts.append(normal((rows, K), w.seed + 7919 + 104729 * i, sd, dt, device))
+    return torch.cat(parts, 0)
+
+
+def segment_offsets(w: Workload):
+    offs = [0]
+    for r in w.segments:
+        offs.append(offs[-1] + r)
+    return offs
+
+
+def sample_rows(M: int, n: int = 256):
+    """Evenly spread row indices, first and last included."""
+    if M <= n:
+        return list(range(M))
+    return sorted({round(i * (M - 1) / (n - 1)) for i in range(n)})
