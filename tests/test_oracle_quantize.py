@@ -209,3 +209,73 @@ def test_tc_layout_roundtrip():
         tc = oracle.scales_to_tc(rm, K)
         assert np.array_equal(oracle.scales_from_tc(tc, R, K), rm)
         assert np.count_nonzero(tc) == rm.size   # padding is zero
+
+
+# ---- FP32 operation order (reading: t = (amax/6)*g and y = x*(g/s)) ----------
+# The pages leave the FP32 evaluation order open.  The orders below differ
+# only near rounding midpoints, so random data rarely tells them apart; these
+# cases are constructed next to E4M3 / E2M1 midpoints, with numpy's IEEE
+# float32 arithmetic as the independent model of each order.
+
+def _find_scale_order_cases(n_want=20):
+    f32 = np.float32
+    vals = E4M3_VALS
+    mids = (vals[8:-1] + vals[9:]) / 2          # midpoints between normal values
+    rng = np.random.default_rng(7)
+    cases = []
+    while len(cases) < n_want:
+        m = mids[rng.integers(0, len(mids))]
+        g = f32(rng.uniform(0.3, 3000.0))
+        a0 = f32(6 * m / np.float64(g))
+        for k in range(-40, 41):
+            a = f32(np.float64(a0) + k * np.spacing(a0))
+            t_ours = f32(f32(a / f32(6)) * g)
+            t_alt = f32(f32(a * g) / f32(6))
+            if oracle.e4m3_encode(t_ours) != oracle.e4m3_encode(t_alt):
+                cases.append((a, g, oracle.e4m3_encode(t_ours)))
+                break
+    return cases
+
+
+def test_scale_op_order_is_amax_over_6_then_times_g():
+    cases = _find_scale_order_cases()
+    assert len(cases) >= 20
+    for a, g, expect in cases:
+        x = np.zeros((1, 16), np.float32)
+        x[0, 3] = a
+        _, scales = oracle.quantize(x, g)
+        assert scales[0, 0] == expect, (a, g)
+
+
+def test_code_op_order_is_x_times_g_over_s():
+    f32 = np.float32
+    rng = np.random.default_rng(8)
+    found = 0
+    tries = 0
+    while found < 20 and tries < 20000:
+        tries += 1
+        g = f32(rng.uniform(0.3, 3000.0))
+        block_max = f32(rng.uniform(0.1, 10.0))
+        s = oracle.e4m3_encode(f32(f32(block_max / f32(6)) * g))
+        if s < 0x08 or s == 0x7E:
+            continue
+        sf = f32(E4M3_VALS[s])
+        mid = rng.choice([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+        x0 = f32(mid * np.float64(sf) / np.float64(g))
+        if x0 >= block_max:
+            continue
+        for k in range(-30, 31):
+            x = f32(np.float64(x0) + k * np.spacing(x0))
+            y_ours = f32(x * f32(g / sf))
+            y_alt = f32(f32(x / sf) * g)
+            c_ours = oracle.e2m1_encode(y_ours)
+            if c_ours != oracle.e2m1_encode(y_alt):
+                blk = np.zeros((1, 16), np.float32)
+                blk[0, 0] = block_max
+                blk[0, 5] = x
+                codes, scales = oracle.quantize(blk, g)
+                assert scales[0, 0] == s
+                assert (codes[0, 2] >> 4) == c_ours, (x, g, block_max)
+                found += 1
+                break
+    assert found >= 20
