@@ -1,0 +1,550 @@
+"""Benchmark of the NVFP4 W4A4 linear layer on B200.
+
+One step = the whole hot path over one batch: quantize the activation to
+NVFP4 (E4M3 block scales, static calibrated global scale), block-scaled
+FP4 GEMM against a pre-quantized weight, dequantizing BF16 epilogue.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode]
+                    [--impl reference] [--no-extra] [--no-cpu-baseline]
+
+The headline line is the decode-shape linear (X[8,5120] x W[12288,5120],
+HBM-bound, GB/s).  Prefill (32768x17408x5120, TFLOP/s), the fused GDN
+projection and the quantize sweep are measured too and reported under
+"extra".  Inputs are seeded synthetic tensors already resident in HBM; the
+decode weight rotates through enough copies to exceed 3x the L2 size, so
+no step reads a weight left in L2 by the previous step.
+
+Multi-GPU (torchrun): every rank runs its own replica on its own batch (the
+layer has no exchange step); value = all ranks' bytes / max-over-ranks time.
+``--impl reference`` times the CPU oracle (the plain C reference) on the
+host on the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 W4A4 GEMM TFLOPS (prefill) & GB/s (decode) vs B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_OVER_BF16 = 4.0          # nominal dense FP4 : BF16 tensor throughput (9 : 2.25 PFLOP/s)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("gemm.cu", "quantize.cu", "ptx.cuh", "common.h", "runtime.cu"):
+        with open(os.path.join(ROOT, "nvfp4_w4a4_quantized_10_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu capture, if it was taken
+    on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        e = t[f"{kernel}:{workload}"]
+        if e.get("source_hash") == source_hash():
+            return e["dram_bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.t is not None:
+            self.t.join(timeout=2)
+
+    def summary(self, t0: float, t1: float):
+        rows = [l for (t, l) in self.lines if t0 - 0.25 <= t <= t1 + 0.25] or [l for (_, l) in self.lines]
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            f = [x.strip() for x in r.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- workloads
+
+class Decode:
+    """Decode-shape linear: X[8,5120] bf16 (0.1 % channels x60), W[12288,5120]."""
+
+    def __init__(self, torch, nv, synth, dev, rank, l2_bytes):
+        w = synth.DECODE
+        self.w = w
+        self.torch, self.nv = torch, nv
+        x = synth.activation(w, device=dev, seed=w.seed + 1000 * rank)
+        wt = synth.weight(w, device=dev)
+        am = torch.empty(1, dtype=torch.float32, device=dev)
+        nv.nvfp4_amax(x, am)
+        self.ga = 2688.0 / am.item()          # static (calibrated) activation scale
+        nv.nvfp4_amax(wt, am)
+        self.gw = 2688.0 / am.item()
+        wc, ws = nv.alloc_quantized(w.N, w.K, dev)
+        nv.nvfp4_quantize(wt, self.gw, wc, ws)
+        per_copy = wc.numel() + ws.numel()
+        self.n_copies = max(2, math.ceil(3 * l2_bytes / per_copy))
+        self.w_copies = [(wc, ws)] + [(wc.clone(), ws.clone()) for _ in range(self.n_copies - 1)]
+        self.x = x
+        self.a_codes, self.a_sc = nv.alloc_quantized(w.M, w.K, dev)
+        self.out = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev)
+        del wt
+        # algorithmic bytes: quantize (X read, codes + scales written) +
+        # GEMM (A codes/scales, W codes/scales read, output written)
+        M, N, K = w.M, w.N, w.K
+        self.gemm_bytes = M * K // 2 + M * K // 16 + N * K // 2 + N * K // 16 + M * N * 2
+        self.quant_bytes = M * K * 2 + M * K // 2 + M * K // 16
+        self.step_bytes = self.gemm_bytes + self.quant_bytes
+        self.launches_per_step = 2
+
+    def step(self, i):
+        nv = self.nv
+        w = self.w
+        wc, ws = self.w_copies[i % self.n_copies]
+        nv.nvfp4_quantize(self.x, self.ga, self.a_codes, self.a_sc)
+        nv.nvfp4_gemm(self.a_codes, self.a_sc, self.ga, wc, ws, self.gw, w.M, w.N, w.K, self.out)
+
+    def gemm_only(self, i):
+        w = self.w
+        wc, ws = self.w_copies[i % self.n_copies]
+        self.nv.nvfp4_gemm(self.a_codes, self.a_sc, self.ga, wc, ws, self.gw, w.M, w.N, w.K, self.out)
+
+    def config(self):
+        w = self.w
+        return {"workload": "decode-shape linear X[8,5120] bf16 x W[12288,5120] nvfp4 -> bf16",
+                "M": w.M, "N": w.N, "K": w.K, "global_batch": w.M,
+                "l2": f"weight rotates through {self.n_copies} copies "
+                      f"({self.n_copies * (w.N * w.K // 2 + w.N * w.K // 16) / 1e6:.0f} MB > 3x L2)"}
+
+
+class Prefill:
+    """Prefill-shape linear: X[32768,5120] heavy-tailed bf16, W[17408,5120]."""
+
+    def __init__(self, torch, nv, synth, dev, rank, l2_bytes, w=None):
+        w = synth.PREFILL if w is None else w
+        self.w = w
+        self.torch, self.nv = torch, nv
+        x = synth.activation(w, device=dev, seed=w.seed + 1000 * rank)
+        wt = synth.weight(w, device=dev)
+        am = torch.empty(1, dtype=torch.float32, device=dev)
+        nv.nvfp4_amax(x, am)
+        self.ga = 2688.0 / am.item()
+        nv.nvfp4_amax(wt, am)
+        self.gw = 2688.0 / am.item()
+        self.wc, self.ws = nv.alloc_quantized(w.N, w.K, dev)
+        nv.nvfp4_quantize(wt, self.gw, self.wc, self.ws)
+        del wt
+        self.x = x
+        self.a_codes, self.a_sc = nv.alloc_quantized(w.M, w.K, dev)
+        self.out = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev)
+        M, N, K = w.M, w.N, w.K
+        self.flops = 2.0 * M * N * K
+        self.launches_per_step = 2
+
+    def step(self, i):
+        w = self.w
+        self.nv.nvfp4_quantize(self.x, self.ga, self.a_codes, self.a_sc)
+        self.nv.nvfp4_gemm(self.a_codes, self.a_sc, self.ga, self.wc, self.ws, self.gw, w.M, w.N, w.K, self.out)
+
+    def gemm_only(self, i):
+        w = self.w
+        self.nv.nvfp4_gemm(self.a_codes, self.a_sc, self.ga, self.wc, self.ws, self.gw, w.M, w.N, w.K, self.out)
+
+
+class FusedGDN:
+    """Fused GDN in-projection: X[4096,5120]; W segments 8192/4096/48/48."""
+
+    def __init__(self, torch, nv, synth, dev, rank, l2_bytes):
+        w = synth.FUSED_GDN
+        self.w = w
+        self.nv = nv
+        x = synth.activation(w, device=dev, seed=w.seed + 1000 * rank)
+        wt = synth.weight(w, device=dev)
+        self.offs = synth.segment_offsets(w)
+        am = torch.empty(1, dtype=torch.float32, device=dev)
+        nv.nvfp4_amax(x, am)
+        self.ga = 2688.0 / am.item()
+        self.gs = []
+        rm = torch.empty(w.N, w.K // 16, dtype=torch.uint8, device=dev)
+        self.wc = torch.empty(w.N, w.K // 2, dtype=torch.uint8, device=dev)
+        for i in range(len(w.segments)):
+            seg = wt[self.offs[i]:self.offs[i + 1]].contiguous()
+            nv.nvfp4_amax(seg, am)
+            g = 2688.0 / am.item()
+            self.gs.append(g)
+            c, s = nv.alloc_quantized(seg.shape[0], w.K, dev, nv.SF_ROWMAJOR)
+            nv.nvfp4_quantize(seg, g, c, s, nv.SF_ROWMAJOR)
+            self.wc[self.offs[i]:self.offs[i + 1]] = c
+            rm[self.offs[i]:self.offs[i + 1]] = s.view(-1, w.K // 16)
+        self.ws = torch.empty(nv.nvfp4_scale_bytes(w.N, w.K), dtype=torch.uint8, device=dev)
+        nv.nvfp4_swizzle_scales(rm, w.N, w.K, self.ws)
+        del wt
+        self.x = x
+        self.a_codes, self.a_sc = nv.alloc_quantized(w.M, w.K, dev)
+        self.out = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev)
+        self.flops = 2.0 * w.M * w.N * w.K
+        self.launches_per_step = 2
+
+    def step(self, i):
+        w = self.w
+        self.nv.nvfp4_quantize(self.x, self.ga, self.a_codes, self.a_sc)
+        self.nv.nvfp4_fused_proj(self.a_codes, self.a_sc, self.ga, self.wc, self.ws, self.offs, self.gs,
+                                 w.M, w.K, self.out)
+
+
+class QuantSweep:
+    def __init__(self, torch, nv, synth, dev, M, K):
+        self.nv = nv
+        self.x = synth.quant_sweep_activation(M, K, device=dev)
+        self.M, self.K = M, K
+        self.codes, self.sc = nv.alloc_quantized(M, K, dev)
+        self.am = torch.empty(1, dtype=torch.float32, device=dev)
+        nv.nvfp4_amax(self.x, self.am)
+        self.g = 2688.0 / self.am.item()
+        self.bytes = M * K * 2 + M * K // 2 + M * K // 16
+
+    def step(self, i):
+        self.nv.nvfp4_quantize(self.x, self.g, self.codes, self.sc, self.nv.SF_TCGEN05, self.am)
+
+
+# ----------------------------------------------------------------- timing
+
+def time_graph(torch, fn, steps, warmup, stream, flush=None):
+    """Warm up eagerly, capture `steps` calls of fn(i) in one CUDA graph,
+    replay once untimed, then time one replay with events on `stream`.
+    Returns (ms per step, graph)."""
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(steps):
+            fn(i)
+    g.replay()
+    torch.cuda.synchronize()
+    if flush is not None:
+        flush()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    g.replay()
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end) / steps, g
+
+
+def time_eager(torch, fn, steps, warmup):
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(s)
+    for i in range(steps):
+        fn(i)
+    end.record(s)
+    end.synchronize()
+    return start.elapsed_time(end) / steps
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+def oracle_decode_sample(budget_s=12.0, max_steps=40):
+    """Time the CPU oracle on the decode workload: quantize X + FP64 GEMM."""
+    import numpy as np
+    import torch
+    import oracle
+    import synth
+    w = synth.DECODE
+    threads = os.cpu_count() or 1
+    oracle.set_threads(threads)
+    x = synth.activation(w).float().numpy()
+    wt = synth.weight(w).float().numpy()
+    gw = oracle.global_scale(oracle.amax(wt))
+    wc, wsc = oracle.quantize(wt, gw)
+    ga = oracle.global_scale(oracle.amax(x))
+    times = []
+    t_end = time.time() + budget_s
+    while len(times) < max_steps and (not times or time.time() < t_end):
+        t0 = time.perf_counter()
+        ac, asc = oracle.quantize(x, ga)
+        oracle.gemm(ac, asc, ga, wc, wsc, gw)
+        times.append(time.perf_counter() - t0)
+    M, N, K = w.M, w.N, w.K
+    step_bytes = (M * K // 2 + M * K // 16 + N * K // 2 + N * K // 16 + M * N * 2) + (M * K * 2 + M * K // 2 + M * K // 16)
+    sec = sum(times) / len(times)
+    return {"value": step_bytes / sec / 1e9, "unit": "GB/s", "cores": oracle.get_threads(), "kind": "oracle",
+            "sample": f"{len(times)} full decode steps (quantize X[8,5120] + FP64 GEMM 8x12288x5120), "
+                      f"{sec * 1e3:.1f} ms each"}, len(times), sec
+
+
+# ----------------------------------------------------------------- ranks
+
+def aggregate_replicas(ms_local: float, units_per_rank: float, world: int, dist=None, device="cpu"):
+    """N independent replicas: the job's time is the slowest rank's, and the
+    job processed world * units_per_rank units in it.  Returns (ms, units/s)."""
+    ms = ms_local
+    if dist is not None and world > 1:
+        import torch
+        t = torch.tensor([ms_local], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms, world * units_per_rank / (ms * 1e-3)
+
+
+# ----------------------------------------------------------------- main
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cpu, n, sec = oracle_decode_sample(budget_s=min(60.0, 6.0 * max(1, args.steps)), max_steps=max(1, args.steps))
+    line = {"impl": "reference", "metric": METRIC, "value": cpu["value"], "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": n, "warmup": 0, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64 (GEMM) / f32 (quantize)", "data": "synthetic",
+            "config": {"workload": "decode-shape linear X[8,5120] bf16 x W[12288,5120] nvfp4 -> bf16",
+                       "M": 8, "N": 12288, "K": 5120, "parallelism": "host cores"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": cpu["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import nvfp4_w4a4_quantized_10_b200 as nv
+    import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(v: float) -> float:
+        return aggregate_replicas(v, 0.0, world, pg, dev)[0]
+
+    peaks, peak_kind = load_peaks()
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 126 * 1024 * 1024) or 126 * 1024 * 1024
+    sampler = ClockSampler(local)
+    sampler.start()
+    stream = torch.cuda.Stream(device=dev)
+
+    # ---- headline: decode step
+    d = Decode(torch, nv, synth, dev, rank, l2)
+    torch.cuda.synchronize()
+    # soak so the clock sampler sees the GPU under this load
+    t_soak = time.time()
+    i = 0
+    while time.time() - t_soak < 1.0:
+        d.step(i)
+        i += 1
+        if i % 64 == 0:
+            torch.cuda.synchronize()
+    barrier()
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        ms_step, g_step = time_graph(torch, d.step, args.steps, args.warmup, stream)
+        ms_gemm, g_gemm = time_graph(torch, d.gemm_only, args.steps, args.warmup, stream)
+    barrier()
+    t1 = time.time()
+    ms_step = max_over_ranks(ms_step)
+    ms_gemm = max_over_ranks(ms_gemm)
+    del g_step, g_gemm
+
+    # ---- end to end through the public API: pinned host X in, host result out
+    x_host = d.x.cpu().pin_memory()
+    out_host = torch.empty(d.out.shape, dtype=d.out.dtype).pin_memory()
+    x_dev = torch.empty_like(d.x)
+
+    def e2e_step(i):
+        x_dev.copy_(x_host, non_blocking=True)
+        wc, ws = d.w_copies[i % d.n_copies]
+        nv.nvfp4_quantize(x_dev, d.ga, d.a_codes, d.a_sc)
+        nv.nvfp4_gemm(d.a_codes, d.a_sc, d.ga, wc, ws, d.gw, d.w.M, d.w.N, d.w.K, d.out)
+        out_host.copy_(d.out, non_blocking=True)
+
+    barrier()
+    ms_e2e = max_over_ranks(time_eager(torch, e2e_step, args.steps, args.warmup))
+    barrier()
+
+    value = aggregate_replicas(ms_step, d.step_bytes, world)[1] / 1e9
+    gemm_gbs = d.gemm_bytes / (ms_gemm * 1e-3) / 1e9
+    hbm_peak = float(peaks["hbm_gbs"])
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, e4m3 block scales, f32 accumulate, bf16 out)",
+        "data": "synthetic (seeded; decode X N(0,1) with 0.1% channels x60, W N(0,0.02))",
+        "config": dict(d.config(), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+        "roofline": {"bound": "hbm", "kernel": "nvfp4_gemm_kernel<16,swap>", "achieved": gemm_gbs,
+                     "peak": hbm_peak, "unit": "GB/s", "frac": gemm_gbs / hbm_peak,
+                     "peak_kind": f"{peak_kind} copy bandwidth",
+                     "algorithmic_bytes_per_launch": d.gemm_bytes, "ms_per_launch": ms_gemm,
+                     "traffic": profiled_traffic("nvfp4_gemm_kernel", "decode")},
+        "e2e": {"value": world * d.step_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
+                "ms_per_step": ms_e2e, "h2d_bytes_per_step": d.x.numel() * d.x.element_size(),
+                "d2h_bytes_per_step": d.out.numel() * d.out.element_size()},
+        "gpu_launches": d.launches_per_step * args.steps,
+    }
+    clk = sampler.summary(t_soak, t1)
+    del d
+
+    # ---- extra workloads (rank 0 measures them only at N = 1)
+    if not args.no_extra and world == 1:
+        extra = {}
+        p = Prefill(torch, nv, synth, dev, rank, l2)
+        k = max(3, min(args.steps, 20))
+        with torch.cuda.stream(stream):
+            ms_p, g1 = time_graph(torch, p.step, k, 3, stream)
+            ms_pg, g2 = time_graph(torch, p.gemm_only, k, 3, stream)
+        del g1, g2
+        fp4_peak = float(peaks["bf16_tflops"]) * FP4_OVER_BF16
+        fp4_sust = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])) * FP4_OVER_BF16
+        tf = p.flops / (ms_pg * 1e-3) / 1e12
+        extra["prefill"] = {
+            "workload": "prefill-shape linear X[32768,5120] bf16 x W[17408,5120] nvfp4 -> bf16",
+            "step_tflops": p.flops / (ms_p * 1e-3) / 1e12, "ms_per_step": ms_p,
+            "roofline": {"bound": "tensor", "kernel": "nvfp4_gemm_kernel<256>", "achieved": tf,
+                         "peak": fp4_peak, "unit": "TFLOP/s", "frac": tf / fp4_peak,
+                         "frac_of_sustained": tf / fp4_sust,
+                         "peak_kind": f"{peak_kind} bf16 cuBLAS x {FP4_OVER_BF16:g} (nominal fp4/bf16)",
+                         "flops_per_launch": p.flops, "ms_per_launch": ms_pg,
+                         "traffic": profiled_traffic("nvfp4_gemm_kernel", "prefill")},
+            "l2": "inputs 129 MB + 1.14 GB output per step exceed L2"}
+        del p
+        f = FusedGDN(torch, nv, synth, dev, rank, l2)
+        with torch.cuda.stream(stream):
+            ms_f, g3 = time_graph(torch, f.step, k, 3, stream)
+        del g3
+        extra["fused_gdn"] = {"workload": "fused GDN projection X[4096,5120] x W[8192|4096|48|48, 5120]",
+                              "step_tflops": f.flops / (ms_f * 1e-3) / 1e12, "ms_per_step": ms_f}
+        del f
+        sweep = {}
+        for M in synth.QUANT_SWEEP_M:
+            for K in synth.QUANT_SWEEP_K:
+                q = QuantSweep(torch, nv, synth, dev, M, K)
+                kk = max(3, min(args.steps, 50))
+                # rotate nothing: M >= 4096 tensors exceed L2 together with their outputs
+                with torch.cuda.stream(stream):
+                    ms_q, g4 = time_graph(torch, q.step, kk, 3, stream)
+                del g4
+                sweep[f"{M}x{K}"] = {"us": ms_q * 1e3, "GB/s": q.bytes / (ms_q * 1e-3) / 1e9,
+                                     "frac_hbm": q.bytes / (ms_q * 1e-3) / 1e9 / hbm_peak}
+                del q
+        extra["quantize_sweep"] = sweep
+        line["extra"] = extra
+
+    sampler.stop()
+    if clk is not None:
+        line["clocks"] = clk
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu, _, _ = oracle_decode_sample()
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line))
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

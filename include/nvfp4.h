@@ -1,0 +1,191 @@
+/*
+ * nvfp4.h - C ABI of the NVFP4 W4A4 linear-layer library for NVIDIA B200
+ * (sm_100a).
+ *
+ * The library implements the three steps of a W4A4 linear layer described
+ * in the write-ups of "Why Gated DeltaNet Survives 4-Bit Quantization: NVFP4
+ * W4A4 for the Recurrent Half of a Hybrid 27B LLM" (arXiv 2609.04098):
+ *
+ *   1. activation quantization to NVFP4: E2M1 4-bit values, one E4M3 scale
+ *      per 16-element block set from the block maximum divided by 6, one FP32
+ *      scale per tensor [picx.dev summary, "Background"];
+ *   2. a block-scaled FP4 x FP4 GEMM on the tensor cores with FP32
+ *      accumulation and a dequantizing BF16 (or FP32) epilogue [same page,
+ *      "Background": native 4-bit tensor-core GEMMs];
+ *   3. the fused projection: several separately calibrated weights
+ *      concatenated along N in one GEMM, each output segment rescaled by its
+ *      own weight global scale, so the fused result equals the unfused ones
+ *      [anthology record LIT-800, "Standing in the anthology"; cctest.ai
+ *      article, "Main findings"; podcast abstract].
+ *
+ * Conventions shared by every entry point
+ *   - Device pointers are raw CUDA device addresses owned by the caller; the
+ *     library never allocates, frees or retains them.  Host pointers (named
+ *     so below) are read during the call only.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and the call returns once enqueued; nothing synchronizes.
+ *   - Arguments are validated before anything is launched.  A failing check
+ *     returns its status and launches nothing.  Launch failures return
+ *     NVFP4_ERR_CUDA.  Faults found by the kernels themselves (a bounded wait
+ *     that ran out) are recorded in a per-device error word, read back by
+ *     nvfp4_last_device_error().  No exception or abort crosses this ABI.
+ *   - Numbers in the format (readings of the pages, which name the formats
+ *     but not their encodings): E2M1 = OCP FP4 (bit 3 sign, 2 exponent bits
+ *     with bias 1, 1 mantissa bit: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6);
+ *     E4M3 = OCP FP8 E4M3FN (bias 7, max 448).  Both are rounded to nearest,
+ *     ties to even, saturating.  A global scale g multiplies on encode and
+ *     divides on decode: value = e2m1(code) * e4m3(scale) / g.
+ *   - Codes: [rows, K/2] bytes, row-major; element 2j of a row is the low
+ *     nibble of byte j.
+ *   - Block scales come in two layouts (nvfp4_sf_layout):
+ *       NVFP4_SF_ROWMAJOR: [rows, K/16] bytes, row-major.
+ *       NVFP4_SF_TCGEN05 : the order the tensor-core MMA reads.  512-byte
+ *         chunks of 128 rows x 4 scales; chunk (r/128, j/4) starts at byte
+ *         ((r/128) * ceil(K/64) + j/4) * 512 and scale j of row r sits at
+ *         (r%32)*16 + ((r/32)%4)*4 + j%4 inside it.  Rows are padded to a
+ *         multiple of 128 and scale columns to a multiple of 4 with zeros;
+ *         the size is nvfp4_scale_bytes(rows, K, NVFP4_SF_TCGEN05).
+ *     The GEMM entry points take NVFP4_SF_TCGEN05 scales only.
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st* nvfp4_stream_t;
+
+typedef enum nvfp4_status {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1,  /* null pointer, bad size, bad scale, bad enum      */
+  NVFP4_ERR_ALIGNMENT = 2,    /* a device pointer is not 16-byte aligned          */
+  NVFP4_ERR_UNSUPPORTED = 3,  /* not an sm_100 device, or a size beyond limits    */
+  NVFP4_ERR_CUDA = 4,         /* a CUDA runtime/driver call or launch failed      */
+  NVFP4_ERR_TIMEOUT = 5,      /* a kernel's bounded wait ran out (device word)    */
+  NVFP4_ERR_DEVICE = 6        /* a kernel found an out-of-range index (device word) */
+} nvfp4_status;
+
+typedef enum nvfp4_in_dtype { NVFP4_IN_BF16 = 0, NVFP4_IN_F32 = 1 } nvfp4_in_dtype;
+typedef enum nvfp4_out_dtype { NVFP4_OUT_BF16 = 0, NVFP4_OUT_F32 = 1 } nvfp4_out_dtype;
+typedef enum nvfp4_sf_layout { NVFP4_SF_ROWMAJOR = 0, NVFP4_SF_TCGEN05 = 1 } nvfp4_sf_layout;
+
+/* Largest number of output segments nvfp4_fused_proj accepts. */
+#define NVFP4_MAX_SEGMENTS 16
+
+/* Bytes needed for the block scales of a [rows, K] operand in `layout`
+ * (0 if rows < 1 or K is not a positive multiple of 16). */
+NVFP4_API size_t nvfp4_scale_bytes(int64_t rows, int64_t K, nvfp4_sf_layout layout);
+
+/* Per-tensor absolute maximum (the input of the default global-scale
+ * calibration g = 448*6/amax) [picx.dev summary, "Background": one FP32
+ * scale per tensor].
+ *   x        device, [M, K] row-major, bf16 or f32 per `dtype`, 16-B aligned
+ *   amax_out device, one float; overwritten with max |x| (0 for an all-zero
+ *            tensor).  Enqueues a 4-byte memset and one kernel.
+ * Errors: INVALID_ARG (null, M < 1, K < 1), ALIGNMENT, CUDA. */
+NVFP4_API nvfp4_status nvfp4_amax(const void* x, nvfp4_in_dtype dtype, int64_t M, int64_t K,
+                        float* amax_out, nvfp4_stream_t stream);
+
+/* NVFP4 quantization of X [M, K] with a given FP32 global scale
+ * [picx.dev summary, "Background"].  For each block of 16 elements along K:
+ *   amax_b = max |x|;  t = (amax_b / 6) * g  (FP32, in this order);
+ *   s = E4M3(t);  if s == 0 every code is a signed zero, else
+ *   r = g / e4m3(s) and code_i = E2M1(x_i * r)   (FP32 multiply).
+ *   x            device [M, K] bf16/f32, 16-byte aligned; K % 32 == 0
+ *   global_scale host float, finite and > 0 (calibrated; 448*6/amax by default)
+ *   codes        device [M, K/2] bytes, 16-byte aligned (written)
+ *   block_scales device, nvfp4_scale_bytes(M, K, layout) bytes, 16-byte
+ *                aligned (written; TCGEN05 padding is written as zero)
+ *   amax_out     device float or NULL; if given, overwritten with max |x|
+ *                (the same value nvfp4_amax returns) as a side output.
+ * Errors: INVALID_ARG (null, M < 1, K < 32 or K % 32, bad g), ALIGNMENT, CUDA. */
+NVFP4_API nvfp4_status nvfp4_quantize(const void* x, nvfp4_in_dtype dtype, int64_t M, int64_t K,
+                            float global_scale, uint8_t* codes, uint8_t* block_scales,
+                            nvfp4_sf_layout layout, float* amax_out, nvfp4_stream_t stream);
+
+/* Rewrite row-major block scales [rows, K/16] into the TCGEN05 layout (used
+ * once, offline, for weights quantized elsewhere).
+ *   rowmajor device [rows, K/16]; tc device nvfp4_scale_bytes(rows, K, TCGEN05)
+ *   bytes, 16-byte aligned (fully written, padding zero).
+ * Errors: INVALID_ARG (null, rows < 1, K % 16), ALIGNMENT, CUDA. */
+NVFP4_API nvfp4_status nvfp4_swizzle_scales(const uint8_t* rowmajor, int64_t rows, int64_t K, uint8_t* tc,
+                                  nvfp4_stream_t stream);
+
+/* W4A4 GEMM with dequantizing epilogue [picx.dev summary, "Background"]:
+ *   out[m, n] = alpha * sum_b sA[m,b] sW[n,b] sum_{k in b} e2m1(A[m,k]) e2m1(W[n,k])
+ * with alpha = 1 / (a_global_scale * w_global_scale) (rounded once to FP32),
+ * FP32 accumulation on the tensor cores, then one rounding to the output type
+ * (bf16 round-to-nearest-even, or f32).
+ *   a_codes [M, K/2], a_scales TCGEN05 layout for M rows   (activations)
+ *   w_codes [N, K/2], w_scales TCGEN05 layout for N rows   (weight, [out, in])
+ *   out     device [M, N] row-major, bf16 or f32 per out_dtype
+ * All device pointers 16-byte aligned; M, N >= 1; K >= 32, K % 32 == 0;
+ * global scales finite and > 0.
+ * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (device is not sm_100), CUDA. */
+NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float a_global_scale,
+                        const uint8_t* w_codes, const uint8_t* w_scales, float w_global_scale,
+                        int64_t M, int64_t N, int64_t K, void* out, nvfp4_out_dtype out_dtype,
+                        nvfp4_stream_t stream);
+
+/* Fused projection: the GEMM above with W the row-wise concatenation of
+ * n_seg separately calibrated weights; output columns
+ * [seg_offsets[i], seg_offsets[i+1]) are rescaled with
+ * alpha_i = 1 / (a_global_scale * seg_global_scales[i]), so each segment of
+ * the result is bitwise equal to nvfp4_gemm on that segment alone
+ * [anthology record LIT-800, "Standing in the anthology"; cctest.ai article,
+ * "Main findings"].  The activation is quantized once, with one scale.
+ *   seg_offsets       host int64[n_seg + 1]: 0 = o_0 < o_1 < ... < o_n = N
+ *   seg_global_scales host float[n_seg], each finite and > 0
+ *   1 <= n_seg <= NVFP4_MAX_SEGMENTS; other arguments as in nvfp4_gemm.
+ * Errors: as nvfp4_gemm. */
+NVFP4_API nvfp4_status nvfp4_fused_proj(const uint8_t* a_codes, const uint8_t* a_scales, float a_global_scale,
+                              const uint8_t* w_codes, const uint8_t* w_scales,
+                              const int64_t* seg_offsets, const float* seg_global_scales, int n_seg,
+                              int64_t M, int64_t K, void* out, nvfp4_out_dtype out_dtype,
+                              nvfp4_stream_t stream);
+
+/* Element conversions exactly as the quantizer performs them, exposed so the
+ * encoders can be checked exhaustively.
+ *   nvfp4_convert_e4m3: out[i] = E4M3(in[i]) (nearest-even, saturating).
+ *   nvfp4_convert_e2m1: n even; out[j] = E2M1(in[2j]) | E2M1(in[2j+1]) << 4.
+ *   in device float[n]; out device bytes (n or n/2).  NaN inputs: unspecified.
+ * Errors: INVALID_ARG (null, n < 1, odd n for e2m1), CUDA. */
+NVFP4_API nvfp4_status nvfp4_convert_e4m3(const float* in, uint8_t* out, int64_t n, nvfp4_stream_t stream);
+NVFP4_API nvfp4_status nvfp4_convert_e2m1(const float* in, uint8_t* out, int64_t n, nvfp4_stream_t stream);
+
+/* Synchronizes the current device, then returns and clears its device error
+ * word: NVFP4_OK, NVFP4_ERR_TIMEOUT or NVFP4_ERR_DEVICE. */
+NVFP4_API nvfp4_status nvfp4_last_device_error(void);
+
+/* Bound (nanoseconds) on every wait inside this library's kernels on all
+ * later launches from this process; 0 restores the default (2 s). */
+NVFP4_API void nvfp4_set_wait_timeout_ns(uint64_t ns);
+
+/* Test entry for the failure path: launches one CTA that waits on an
+ * mbarrier nothing ever arrives on, bounded by `timeout_ns`.  The kernel
+ * records NVFP4_ERR_TIMEOUT in the device error word and exits; the context
+ * stays usable.  Errors: INVALID_ARG (timeout_ns 0 or above 10 s), CUDA. */
+NVFP4_API nvfp4_status nvfp4_test_wait_timeout(uint64_t timeout_ns, nvfp4_stream_t stream);
+
+/* Static description of a status code. */
+NVFP4_API const char* nvfp4_status_string(nvfp4_status status);
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+NVFP4_API int nvfp4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H_ */

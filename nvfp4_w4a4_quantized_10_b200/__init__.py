@@ -1,0 +1,189 @@
+"""Python binding of the NVFP4 W4A4 linear-layer library (libnvfp4.so).
+
+Argument marshalling only: every function below passes raw device pointers,
+sizes and the current CUDA stream of the given tensors to the C-ABI function
+of the same name (declared in ``include/nvfp4.h``) and raises ``Nvfp4Error``
+on a non-OK status.  All quantization and GEMM work runs in the library's
+CUDA kernels; there is no CPU fallback.  PyTorch supplies device memory and
+streams.
+
+The library is built in-tree by ``python -m nvfp4_w4a4_quantized_10_b200.build``;
+importing this package without it raises ImportError.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libnvfp4.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "nvfp4.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libnvfp4.so is not built ({LIB_PATH}); run "
+                      "`python -m nvfp4_w4a4_quantized_10_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+# status / enums (mirror include/nvfp4.h)
+OK, ERR_INVALID_ARG, ERR_ALIGNMENT, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE = range(7)
+IN_BF16, IN_F32 = 0, 1
+OUT_BF16, OUT_F32 = 0, 1
+SF_ROWMAJOR, SF_TCGEN05 = 0, 1
+MAX_SEGMENTS = 16
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_f32 = ctypes.c_float
+
+_lib.nvfp4_scale_bytes.restype = ctypes.c_size_t
+_lib.nvfp4_scale_bytes.argtypes = [_i64, _i64, ctypes.c_int]
+_lib.nvfp4_amax.argtypes = [_vp, ctypes.c_int, _i64, _i64, _vp, _vp]
+_lib.nvfp4_quantize.argtypes = [_vp, ctypes.c_int, _i64, _i64, _f32, _vp, _vp, ctypes.c_int, _vp, _vp]
+_lib.nvfp4_swizzle_scales.argtypes = [_vp, _i64, _i64, _vp, _vp]
+_lib.nvfp4_gemm.argtypes = [_vp, _vp, _f32, _vp, _vp, _f32, _i64, _i64, _i64, _vp, ctypes.c_int, _vp]
+_lib.nvfp4_fused_proj.argtypes = [_vp, _vp, _f32, _vp, _vp, ctypes.POINTER(_i64), ctypes.POINTER(_f32),
+                                  ctypes.c_int, _i64, _i64, _vp, ctypes.c_int, _vp]
+_lib.nvfp4_convert_e4m3.argtypes = [_vp, _vp, _i64, _vp]
+_lib.nvfp4_convert_e2m1.argtypes = [_vp, _vp, _i64, _vp]
+_lib.nvfp4_last_device_error.argtypes = []
+_lib.nvfp4_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+_lib.nvfp4_set_wait_timeout_ns.restype = None
+_lib.nvfp4_test_wait_timeout.argtypes = [ctypes.c_uint64, _vp]
+_lib.nvfp4_status_string.restype = ctypes.c_char_p
+_lib.nvfp4_status_string.argtypes = [ctypes.c_int]
+_lib.nvfp4_version.restype = ctypes.c_int
+
+
+class Nvfp4Error(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: {status_string(status)} (status {status})")
+
+
+def lib():
+    return _lib
+
+
+def declared_symbols() -> list[str]:
+    """Names of the functions include/nvfp4.h declares."""
+    with open(HEADER) as f:
+        text = f.read()
+    return re.findall(r"NVFP4_API\s+[\w\s\*]+?\b(nvfp4_\w+)\s*\(", text)
+
+
+def status_string(status: int) -> str:
+    return _lib.nvfp4_status_string(int(status)).decode()
+
+
+def version() -> int:
+    return int(_lib.nvfp4_version())
+
+
+def _check(fn, status):
+    if status != OK:
+        raise Nvfp4Error(fn, status)
+
+
+def _stream(t: torch.Tensor):
+    return _vp(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("device tensor expected")
+    if not t.is_contiguous():
+        raise ValueError("contiguous tensor expected")
+    return _vp(t.data_ptr())
+
+
+def _in_dtype(x: torch.Tensor) -> int:
+    if x.dtype == torch.bfloat16:
+        return IN_BF16
+    if x.dtype == torch.float32:
+        return IN_F32
+    raise ValueError(f"unsupported input dtype {x.dtype}")
+
+
+def _out_dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return OUT_BF16
+    if t.dtype == torch.float32:
+        return OUT_F32
+    raise ValueError(f"unsupported output dtype {t.dtype}")
+
+
+# ---------------------------------------------------------------- C-ABI calls
+
+def nvfp4_scale_bytes(rows: int, K: int, layout: int = SF_TCGEN05) -> int:
+    return int(_lib.nvfp4_scale_bytes(rows, K, layout))
+
+
+def nvfp4_amax(x: torch.Tensor, amax_out: torch.Tensor) -> None:
+    M, K = x.shape
+    _check("nvfp4_amax", _lib.nvfp4_amax(_ptr(x), _in_dtype(x), M, K, _ptr(amax_out), _stream(x)))
+
+
+def nvfp4_quantize(x: torch.Tensor, global_scale: float, codes: torch.Tensor, block_scales: torch.Tensor,
+                   layout: int = SF_TCGEN05, amax_out: torch.Tensor | None = None) -> None:
+    M, K = x.shape
+    _check("nvfp4_quantize", _lib.nvfp4_quantize(_ptr(x), _in_dtype(x), M, K, float(global_scale), _ptr(codes),
+                                                 _ptr(block_scales), layout, _ptr(amax_out), _stream(x)))
+
+
+def nvfp4_swizzle_scales(rowmajor: torch.Tensor, rows: int, K: int, tc: torch.Tensor) -> None:
+    _check("nvfp4_swizzle_scales",
+           _lib.nvfp4_swizzle_scales(_ptr(rowmajor), rows, K, _ptr(tc), _stream(tc)))
+
+
+def nvfp4_gemm(a_codes, a_scales, a_global_scale, w_codes, w_scales, w_global_scale, M, N, K,
+               out: torch.Tensor) -> None:
+    _check("nvfp4_gemm", _lib.nvfp4_gemm(_ptr(a_codes), _ptr(a_scales), float(a_global_scale), _ptr(w_codes),
+                                         _ptr(w_scales), float(w_global_scale), M, N, K, _ptr(out),
+                                         _out_dtype(out), _stream(out)))
+
+
+def nvfp4_fused_proj(a_codes, a_scales, a_global_scale, w_codes, w_scales, seg_offsets, seg_global_scales,
+                     M, K, out: torch.Tensor) -> None:
+    n = len(seg_global_scales)
+    offs = (_i64 * (n + 1))(*[int(v) for v in seg_offsets])
+    gs = (_f32 * n)(*[float(v) for v in seg_global_scales])
+    _check("nvfp4_fused_proj",
+           _lib.nvfp4_fused_proj(_ptr(a_codes), _ptr(a_scales), float(a_global_scale), _ptr(w_codes),
+                                 _ptr(w_scales), offs, gs, n, M, K, _ptr(out), _out_dtype(out), _stream(out)))
+
+
+def nvfp4_convert_e4m3(x: torch.Tensor, out: torch.Tensor) -> None:
+    _check("nvfp4_convert_e4m3", _lib.nvfp4_convert_e4m3(_ptr(x), _ptr(out), x.numel(), _stream(x)))
+
+
+def nvfp4_convert_e2m1(x: torch.Tensor, out: torch.Tensor) -> None:
+    _check("nvfp4_convert_e2m1", _lib.nvfp4_convert_e2m1(_ptr(x), _ptr(out), x.numel(), _stream(x)))
+
+
+def nvfp4_last_device_error() -> int:
+    return int(_lib.nvfp4_last_device_error())
+
+
+def nvfp4_set_wait_timeout_ns(ns: int) -> None:
+    _lib.nvfp4_set_wait_timeout_ns(int(ns))
+
+
+def nvfp4_test_wait_timeout(timeout_ns: int, device=None) -> None:
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    _check("nvfp4_test_wait_timeout",
+           _lib.nvfp4_test_wait_timeout(int(timeout_ns), _vp(torch.cuda.current_stream(dev).cuda_stream)))
+
+
+# ---------------------------------------------------------------- buffers
+
+def alloc_quantized(rows: int, K: int, device, layout: int = SF_TCGEN05):
+    """Empty (codes, scales) buffers for a [rows, K] NVFP4 operand."""
+    codes = torch.empty(rows, K // 2, dtype=torch.uint8, device=device)
+    scales = torch.empty(nvfp4_scale_bytes(rows, K, layout), dtype=torch.uint8, device=device)
+    return codes, scales

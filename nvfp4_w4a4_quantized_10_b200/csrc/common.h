@@ -1,0 +1,46 @@
+// Host-side helpers shared by the library's translation units: argument
+// checks, per-device state (error word, SM count, architecture), launch
+// configuration.  No torch types; plain CUDA runtime.
+#pragma once
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/nvfp4.h"
+
+namespace nvfp4 {
+
+struct DeviceInfo {
+  int device = -1;
+  int sm_count = 0;
+  int major = 0, minor = 0;
+  size_t max_smem_optin = 0;
+  unsigned* err_word = nullptr;  // device address of this device's error word
+};
+
+// Per-device information; initialised on first use on the current device.
+// Returns nullptr if the CUDA runtime fails.
+const DeviceInfo* device_info();
+
+// Wait bound for every kernel of the library (ns).
+uint64_t wait_timeout_ns();
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool finite_positive(float g) {
+  uint32_t b;
+  std::memcpy(&b, &g, 4);
+  const bool finite = ((b >> 23) & 0xFF) != 0xFF;
+  return finite && g > 0.0f;
+}
+
+inline nvfp4_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return NVFP4_OK;
+  (void)cudaGetLastError();  // do not leave a sticky launch error for the caller's next check
+  return NVFP4_ERR_CUDA;
+}
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace nvfp4

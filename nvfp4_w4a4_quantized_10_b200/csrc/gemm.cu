@@ -1,0 +1,515 @@
+// Block-scaled NVFP4 x NVFP4 GEMM with a dequantizing epilogue, and the fused
+// multi-segment projection, for sm_100a.
+//
+// What it computes [picx.dev summary of "Why Gated DeltaNet Survives 4-Bit
+// Quantization", "Background": native 4-bit tensor-core GEMMs on NVFP4
+// operands; anthology record LIT-800, "Standing in the anthology", and the
+// cctest.ai article, "Main findings": fused projections must apply each
+// module's own global scale]:
+//   out[m,n] = alpha(n) * sum_b sA[m,b] sW[n,b] sum_{k in b} e2m1(A[m,k]) e2m1(W[n,k])
+//   alpha(n) = 1 / (gA * gW[segment of n])
+//
+// Design (one persistent CTA per SM, 6 warps):
+//   warp 0    TMA producer: per 256-wide K step, one 2-D TMA box of each
+//             operand's codes (128-byte rows, 128B swizzle) and one or two
+//             bulk copies of the pre-swizzled E4M3 scale chunks, all landing
+//             on one mbarrier with an expected byte count.
+//   warp 1    TMEM allocator and MMA issuer: copies the scale chunks from
+//             shared memory into TMEM (tcgen05.cp 32x128b.warpx4), then
+//             issues four tcgen05.mma kind::mxf4nvf4 block_scale (K = 64
+//             each) into the FP32 accumulator in TMEM, and releases the
+//             stage with tcgen05.commit.
+//   warps 2-5 epilogue: tcgen05.ld the accumulator (one TMEM lane per
+//             output row), scale by alpha, round once to bf16 (or keep
+//             f32), free the accumulator, store.
+// Two tile shapes:
+//   normal  P = activations (128-row tiles), Q = weight (256-row tiles):
+//           prefill and fused projections.
+//   swap    P = weight (128-row tiles), Q = all activation rows (<= 128):
+//           decode, so the 128-row MMA dimension walks the weight and the
+//           grid covers N/128 tiles that stream W from HBM.
+// Every mbarrier wait is bounded (see ptx.cuh); on timeout the CTA drains
+// its in-flight copies and MMAs (bounded again), frees TMEM and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <mutex>
+
+#include "common.h"
+#include "ptx.cuh"
+
+namespace nvfp4 {
+
+constexpr int kBM = 128;          // MMA M: rows of operand P per tile
+constexpr int kBKBytes = 128;     // bytes of codes per row per stage (256 elements)
+constexpr int kSfChunk = 512;     // bytes of one 128-row x 4-scale chunk
+constexpr int kThreads = 192;
+constexpr int kTmemCols = 512;
+constexpr int kGroupP = 8;        // tile raster: 8 P-tiles share a Q-tile
+
+struct alignas(64) GemmParams {
+  CUtensorMap tmap_p;
+  CUtensorMap tmap_q;
+  const uint8_t* sf_p;
+  const uint8_t* sf_q;
+  void* out;
+  unsigned* err;
+  uint64_t timeout_ns;
+  int64_t M, N;          // output [M, N]
+  int rows_p, rows_q;    // rows of the P and Q operands
+  int rb_q;              // 128-row scale blocks allocated for Q
+  int kc;                // ceil(K / 64): scale chunks per row block
+  int kt;                // ceil(K / 256): pipeline steps per tile
+  int tiles_p, tiles_q;
+  int n_seg;
+  int seg_end[NVFP4_MAX_SEGMENTS];
+  float seg_alpha[NVFP4_MAX_SEGMENTS];
+};
+
+template <int BN, bool SWAP>
+struct Cfg {
+  static constexpr int kSfbBlocks = (BN + 127) / 128;                // 128-row scale blocks of Q
+  static constexpr int kABytes = kBM * kBKBytes;                     // 16 KB
+  static constexpr int kBBytes = BN * kBKBytes;
+  static constexpr int kSfaBytes = 4 * kSfChunk;                     // 2 KB
+  static constexpr int kSfbBytes = kSfbBlocks * 4 * kSfChunk;
+  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  static constexpr int kMaxStages = SWAP ? 8 : 4;
+  static constexpr int kStages =
+      (220 * 1024) / kStageBytes < kMaxStages ? (220 * 1024) / kStageBytes : kMaxStages;
+  static constexpr int kOffA = 0;
+  static constexpr int kOffB = kOffA + kStages * kABytes;
+  static constexpr int kOffSfa = kOffB + kStages * kBBytes;
+  static constexpr int kOffSfb = kOffSfa + kStages * kSfaBytes;
+  static constexpr int kOffBar = kOffSfb + kStages * kSfbBytes;
+  static constexpr int kNumBars = 2 * kStages + 3;                   // full, empty, acc_full, acc_empty, drain
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;            // + alignment slack
+  // TMEM columns: accumulator, then per-stage scale regions
+  static constexpr int kAccCols = BN < 32 ? 32 : BN;
+  static constexpr int kSfaCols = 16;                                // 4 MMAs x 4 columns
+  static constexpr int kSfbCols = kSfbBlocks * 16;
+  static constexpr int kSfStageCols = kSfaCols + kSfbCols;
+  static_assert(kAccCols + kStages * kSfStageCols <= kTmemCols, "TMEM budget");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(BN % 16 == 0 && BN <= 256, "MMA N");
+};
+
+__device__ __forceinline__ int seg_index(const GemmParams& p, int64_t n) {
+  int i = 0;
+  while (i < p.n_seg - 1 && n >= p.seg_end[i]) ++i;
+  return i;
+}
+
+__device__ __forceinline__ float seg_alpha(const GemmParams& p, int64_t n) { return p.seg_alpha[seg_index(p, n)]; }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);   // round to nearest even
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void tile_coords(const GemmParams& p, int tile, int& tp, int& tq) {
+  const int per_group = kGroupP * p.tiles_q;
+  const int group = tile / per_group;
+  const int first = group * kGroupP;
+  const int gsize = min(p.tiles_p - first, kGroupP);
+  const int local = tile - group * per_group;
+  tp = first + local % gsize;
+  tq = local / gsize;
+}
+
+template <int BN, bool SWAP, bool OUT_F32>
+__global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_constant__ GemmParams p) {
+  using C = Cfg<BN, SWAP>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar_full = sbase + C::kOffBar;
+  const uint32_t bar_empty = bar_full + 8 * C::kStages;
+  const uint32_t bar_acc_full = bar_empty + 8 * C::kStages;
+  const uint32_t bar_acc_empty = bar_acc_full + 8;
+  const uint32_t bar_drain = bar_acc_empty + 8;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int total_tiles = p.tiles_p * p.tiles_q;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    mbar_init(bar_acc_full, 1);
+    mbar_init(bar_acc_empty, 128);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&p.tmap_p);
+    prefetch_tmap(&p.tmap_q);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, last_parity = 0;   // for the drain on abort
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+        int tp, tq;
+        tile_coords(p, tile, tp, tq);
+        const int p0 = tp * kBM, q0 = tq * BN;
+        const uint8_t* sfp = p.sf_p + (size_t)(p0 >> 7) * p.kc * kSfChunk;
+        for (int k = 0; k < p.kt; ++k) {
+          if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, p.err, p.timeout_ns)) { ok = false; break; }
+          const int nch = min(4, p.kc - 4 * k);
+          const uint32_t sf_bytes = (uint32_t)nch * kSfChunk;
+          int nsfb = 0;
+#pragma unroll
+          for (int rb = 0; rb < C::kSfbBlocks; ++rb)
+            if ((q0 >> 7) + rb < p.rb_q) ++nsfb;
+          const uint32_t fb = bar_full + 8 * stage;
+          mbar_arrive_expect_tx(fb, C::kABytes + C::kBBytes + sf_bytes * (1 + nsfb));
+          tma_load_2d(sbase + C::kOffA + stage * C::kABytes, &p.tmap_p, k * kBKBytes, p0, fb);
+          tma_load_2d(sbase + C::kOffB + stage * C::kBBytes, &p.tmap_q, k * kBKBytes, q0, fb);
+          bulk_load(sbase + C::kOffSfa + stage * C::kSfaBytes, sfp + (size_t)(4 * k) * kSfChunk, sf_bytes, fb);
+#pragma unroll
+          for (int rb = 0; rb < C::kSfbBlocks; ++rb) {
+            const int qb = (q0 >> 7) + rb;
+            if (qb < p.rb_q)
+              bulk_load(sbase + C::kOffSfb + stage * C::kSfbBytes + rb * 4 * kSfChunk,
+                        p.sf_q + ((size_t)qb * p.kc + 4 * k) * kSfChunk, sf_bytes, fb);
+          }
+          issued_mask |= 1u << stage;
+          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (*abort_flag) {
+        // let every issued copy land before the CTA exits
+        for (int s = 0; s < C::kStages; ++s)
+          if (issued_mask & (1u << s)) {
+            volatile int never = 0;
+            (void)mbar_wait(bar_full + 8 * s, (last_parity >> s) & 1, &never, p.err, p.timeout_ns);
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_nvf4(kBM, BN);
+      const uint32_t acc = tmem_base;
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(bar_acc_empty, acc_phase ^ 1, abort_flag, p.err, p.timeout_ns)) break;
+        tc_fence_after();
+        for (int k = 0; k < p.kt; ++k) {
+          if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, p.err, p.timeout_ns)) { ok = false; break; }
+          tc_fence_after();
+          const int nkb = min(4, p.kc - 4 * k);
+          const uint32_t sfa_t = tmem_base + C::kAccCols + stage * C::kSfStageCols;
+          const uint32_t sfb_t = sfa_t + C::kSfaCols;
+          const uint32_t sa = sbase + C::kOffSfa + stage * C::kSfaBytes;
+          const uint32_t sb = sbase + C::kOffSfb + stage * C::kSfbBytes;
+          for (int kb = 0; kb < nkb; ++kb) {
+            // 32 rows x 16 bytes, core matrices of 8 rows 128 bytes apart
+            tc_cp_32x128b_warpx4(sfa_t + kb * 4, smem_desc(sa + kb * kSfChunk, 16, 128, 0));
+#pragma unroll
+            for (int rb = 0; rb < C::kSfbBlocks; ++rb)
+              tc_cp_32x128b_warpx4(sfb_t + kb * 4 * C::kSfbBlocks + rb * 4,
+                                   smem_desc(sb + rb * 4 * kSfChunk + kb * kSfChunk, 16, 128, 0));
+          }
+          const uint32_t a_s = sbase + C::kOffA + stage * C::kABytes;
+          const uint32_t b_s = sbase + C::kOffB + stage * C::kBBytes;
+          for (int kb = 0; kb < nkb; ++kb) {
+            // K-major, 128B swizzle: 8-row groups 1024 bytes apart; a K step
+            // of 64 FP4 elements is 32 bytes inside the swizzle atom
+            const uint64_t ad = smem_desc(a_s + kb * 32, 16, 1024, 2);
+            const uint64_t bd = smem_desc(b_s + kb * 32, 16, 1024, 2);
+            tc_mma_nvf4(acc, ad, bd, idesc, sfa_t + kb * 4, sfb_t + kb * 4 * C::kSfbBlocks,
+                        (k | kb) != 0 ? 1u : 0u);
+          }
+          tc_commit(bar_empty + 8 * stage);
+          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        tc_commit(bar_acc_full);
+        acc_phase ^= 1;
+      }
+      // every MMA and scale copy issued by this thread has completed once
+      // this commit arrives
+      tc_commit(bar_drain);
+      volatile int never = 0;
+      (void)mbar_wait(bar_drain, 0, &never, p.err, p.timeout_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int sp = warp & 3;                 // TMEM subpartition of this warp
+    const int row = sp * 32 + lane;          // accumulator lane = tile row of P
+    const uint32_t taddr = tmem_base + ((uint32_t)(sp * 32) << 16);
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      int tp, tq;
+      tile_coords(p, tile, tp, tq);
+      const int64_t p0 = (int64_t)tp * kBM, q0 = (int64_t)tq * BN;
+      if (!mbar_wait(bar_acc_full, acc_phase, abort_flag, p.err, p.timeout_ns)) break;
+      __syncwarp();
+      tc_fence_after();
+      if constexpr (!SWAP) {
+        const int64_t m = p0 + row;
+        if constexpr (!OUT_F32) {
+          uint32_t packed[BN / 2];
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(taddr + c * 32, r);
+            tmem_ld_wait();
+            const int64_t nb = q0 + c * 32;
+            const bool uniform = seg_index(p, nb) == seg_index(p, nb + 31);
+            const float a0 = seg_alpha(p, nb);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float alo = uniform ? a0 : seg_alpha(p, nb + 2 * i);
+              const float ahi = uniform ? a0 : seg_alpha(p, nb + 2 * i + 1);
+              packed[c * 16 + i] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * i]), alo),
+                                               __fmul_rn(__uint_as_float(r[2 * i + 1]), ahi));
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(bar_acc_empty);
+          if (m < p.M) {
+            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + m * p.N;
+            const bool vec = (p.N % 8) == 0;
+#pragma unroll
+            for (int c = 0; c < BN / 8; ++c) {
+              const int64_t n = q0 + c * 8;
+              if (vec && n + 8 <= p.N) {
+                *reinterpret_cast<uint4*>(orow + n) =
+                    make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+              } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                  if (n + e < p.N)
+                    reinterpret_cast<uint16_t*>(orow)[n + e] =
+                        (uint16_t)(packed[4 * c + e / 2] >> (16 * (e & 1)));
+              }
+            }
+          }
+        } else {
+          float* orow = reinterpret_cast<float*>(p.out) + m * p.N;
+#pragma unroll 1
+          for (int c = 0; c < BN / 32; ++c) {
+            uint32_t r[32];
+            __syncwarp();
+            tmem_ld_32x32b_x32(taddr + c * 32, r);
+            tmem_ld_wait();
+            if (m < p.M) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const int64_t n = q0 + c * 32 + i;
+                if (n < p.N) orow[n] = __fmul_rn(__uint_as_float(r[i]), seg_alpha(p, n));
+              }
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(bar_acc_empty);
+        }
+      } else {
+        // swap: lane = weight row = output column n; accumulator column = activation row
+        const int64_t n = p0 + row;
+        const float alpha = seg_alpha(p, n);
+#pragma unroll
+        for (int c = 0; c < (BN + 31) / 32; ++c) {
+          uint32_t r[32];
+          __syncwarp();
+          if constexpr (BN >= 32) {
+            tmem_ld_32x32b_x32(taddr + c * 32, r);
+          } else {
+            uint32_t r8[8];
+#pragma unroll
+            for (int j = 0; j < BN / 8; ++j) {
+              tmem_ld_32x32b_x8(taddr + j * 8, r8);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) r[j * 8 + i] = r8[i];
+            }
+          }
+          tmem_ld_wait();
+          if (n < p.N) {
+#pragma unroll
+            for (int i = 0; i < (BN < 32 ? BN : 32); ++i) {
+              const int64_t m = q0 + c * 32 + i;
+              if (m < p.M) {
+                const float v = __fmul_rn(__uint_as_float(r[i]), alpha);
+                if constexpr (OUT_F32) reinterpret_cast<float*>(p.out)[m * p.N + n] = v;
+                else reinterpret_cast<__nv_bfloat16*>(p.out)[m * p.N + n] = __float2bfloat16_rn(v);
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar_acc_empty);
+      }
+      acc_phase ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+    else
+      (void)cudaGetLastError();
+  });
+  return fn;
+}
+
+// Codes of a [rows, K/2]-byte operand, 128-byte x box_rows boxes, 128B swizzle.
+bool make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+  const cuuint32_t box[2] = {(cuuint32_t)kBKBytes, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, bool SWAP, bool OUT_F32>
+cudaError_t launch(const GemmParams& p, const DeviceInfo* d, cudaStream_t st) {
+  using Cf = Cfg<BN, SWAP>;
+  auto kern = nvfp4_gemm_kernel<BN, SWAP, OUT_F32>;
+  static std::once_flag once[64];
+  static cudaError_t attr_err[64];
+  std::call_once(once[d->device], [&] {
+    attr_err[d->device] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmemBytes);
+  });
+  if (attr_err[d->device] != cudaSuccess) return attr_err[d->device];
+  const int tiles = p.tiles_p * p.tiles_q;
+  const int grid = tiles < d->sm_count ? tiles : d->sm_count;
+  kern<<<grid, kThreads, Cf::kSmemBytes, st>>>(p);
+  return cudaGetLastError();
+}
+
+float alpha_of(float ga, float gw) { return (float)(1.0 / ((double)ga * (double)gw)); }
+
+nvfp4_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float ga, const uint8_t* w_codes,
+                      const uint8_t* w_scales, const int64_t* seg_offsets, const float* seg_gs, int n_seg,
+                      int64_t M, int64_t N, int64_t K, void* out, nvfp4_out_dtype out_dtype, cudaStream_t st) {
+  if (!a_codes || !a_scales || !w_codes || !w_scales || !out) return NVFP4_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 32 || K % 32 != 0) return NVFP4_ERR_INVALID_ARG;
+  if (M > (1ll << 31) - 256 || N > (1ll << 31) - 256 || K > (1ll << 31)) return NVFP4_ERR_UNSUPPORTED;
+  if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F32) return NVFP4_ERR_INVALID_ARG;
+  if (!finite_positive(ga)) return NVFP4_ERR_INVALID_ARG;
+  if (n_seg < 1 || n_seg > NVFP4_MAX_SEGMENTS) return NVFP4_ERR_INVALID_ARG;
+  for (int i = 0; i < n_seg; ++i)
+    if (!finite_positive(seg_gs[i]) || seg_offsets[i + 1] <= seg_offsets[i]) return NVFP4_ERR_INVALID_ARG;
+  if (seg_offsets[0] != 0 || seg_offsets[n_seg] != N) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
+      !aligned16(out))
+    return NVFP4_ERR_ALIGNMENT;
+  const DeviceInfo* d = device_info();
+  if (!d) return NVFP4_ERR_CUDA;
+  if (d->major != 10) return NVFP4_ERR_UNSUPPORTED;
+
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  const bool swap = M <= 128;
+  int bn = 256;
+  if (swap) bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+  p.rows_p = (int)(swap ? N : M);
+  p.rows_q = (int)(swap ? M : N);
+  const uint8_t* codes_p = swap ? w_codes : a_codes;
+  const uint8_t* codes_q = swap ? a_codes : w_codes;
+  p.sf_p = swap ? w_scales : a_scales;
+  p.sf_q = swap ? a_scales : w_scales;
+  if (!make_code_map(&p.tmap_p, codes_p, p.rows_p, K, kBM) || !make_code_map(&p.tmap_q, codes_q, p.rows_q, K, bn))
+    return NVFP4_ERR_CUDA;
+  p.out = out;
+  p.err = d->err_word;
+  p.timeout_ns = wait_timeout_ns();
+  p.M = M;
+  p.N = N;
+  p.rb_q = (int)ceil_div(p.rows_q, 128);
+  p.kc = (int)ceil_div(K, 64);
+  p.kt = (int)ceil_div(K, 256);
+  p.tiles_p = (int)ceil_div(p.rows_p, kBM);
+  p.tiles_q = (int)ceil_div(p.rows_q, bn);
+  p.n_seg = n_seg;
+  for (int i = 0; i < n_seg; ++i) {
+    p.seg_end[i] = (int)seg_offsets[i + 1];
+    p.seg_alpha[i] = alpha_of(ga, seg_gs[i]);
+  }
+  const bool f32 = out_dtype == NVFP4_OUT_F32;
+  cudaError_t e;
+  if (!swap) e = f32 ? launch<256, false, true>(p, d, st) : launch<256, false, false>(p, d, st);
+  else if (bn == 16) e = f32 ? launch<16, true, true>(p, d, st) : launch<16, true, false>(p, d, st);
+  else if (bn == 32) e = f32 ? launch<32, true, true>(p, d, st) : launch<32, true, false>(p, d, st);
+  else if (bn == 64) e = f32 ? launch<64, true, true>(p, d, st) : launch<64, true, false>(p, d, st);
+  else e = f32 ? launch<128, true, true>(p, d, st) : launch<128, true, false>(p, d, st);
+  return cuda_status(e);
+}
+
+}  // namespace
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+extern "C" {
+
+nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float a_global_scale,
+                        const uint8_t* w_codes, const uint8_t* w_scales, float w_global_scale, int64_t M, int64_t N,
+                        int64_t K, void* out, nvfp4_out_dtype out_dtype, nvfp4_stream_t stream) {
+  const int64_t offs[2] = {0, N};
+  const float gs[1] = {w_global_scale};
+  return run_gemm(a_codes, a_scales, a_global_scale, w_codes, w_scales, offs, gs, 1, M, N, K, out, out_dtype,
+                  (cudaStream_t)stream);
+}
+
+nvfp4_status nvfp4_fused_proj(const uint8_t* a_codes, const uint8_t* a_scales, float a_global_scale,
+                              const uint8_t* w_codes, const uint8_t* w_scales, const int64_t* seg_offsets,
+                              const float* seg_global_scales, int n_seg, int64_t M, int64_t K, void* out,
+                              nvfp4_out_dtype out_dtype, nvfp4_stream_t stream) {
+  if (!seg_offsets || !seg_global_scales || n_seg < 1 || n_seg > NVFP4_MAX_SEGMENTS) return NVFP4_ERR_INVALID_ARG;
+  return run_gemm(a_codes, a_scales, a_global_scale, w_codes, w_scales, seg_offsets, seg_global_scales, n_seg, M,
+                  seg_offsets[n_seg], K, out, out_dtype, (cudaStream_t)stream);
+}
+
+}  // extern "C"

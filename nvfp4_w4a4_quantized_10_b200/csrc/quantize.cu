@@ -1,0 +1,379 @@
+// NVFP4 activation quantization, per-tensor amax, scale-layout rewrite and
+// the element conversions.
+//
+// Format [picx.dev summary of "Why Gated DeltaNet Survives 4-Bit
+// Quantization", "Background"]: E2M1 values, one E4M3 scale per 16-element
+// block set from blockmax/6, one FP32 scale per tensor.  Per block:
+//   amax_b = max|x|, t = (amax_b/6)*g, s = E4M3_rn_sat(t),
+//   s == 0 -> signed-zero codes, else r = g/e4m3(s), code = E2M1_rn_sat(x*r).
+// All FP32 steps use explicitly rounded intrinsics (no contraction), and the
+// FP8/FP4 encodings use the hardware cvt.rn.satfinite conversions.
+//
+// Work split: two adjacent threads own one 16-element block (8 elements, one
+// 16-byte bf16 load each), exchange their half maxima with one shuffle, and
+// each writes 4 bytes of codes, so a warp reads 512 contiguous bytes and
+// writes 128 contiguous bytes.  The kernel is HBM-bound (2.5625 bytes per
+// bf16 element); four independent loads per thread are in flight per
+// iteration.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "common.h"
+#include "ptx.cuh"
+
+namespace nvfp4 {
+
+// ----------------------------------------------------------------- encoders
+
+__device__ __forceinline__ uint32_t cvt_e4m3(float t) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(t), "f"(t));
+  return r & 0xFFu;
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint32_t s) {
+  uint32_t h2;
+  const uint16_t in = (uint16_t)(s & 0xFF);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFF)));
+}
+
+// Eight floats -> eight E2M1 codes, element 0 in the low nibble of the low byte.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&y)[8]) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]), "f"(y[7]));
+  return out;
+}
+
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.u32.u8 %0, b0;\n\t}"
+      : "=r"(out)
+      : "f"(lo), "f"(hi));
+  return out;
+}
+
+// Offset of scale j of row r in the tensor-core scale layout.
+__device__ __forceinline__ int64_t tc_scale_offset(int64_t r, int64_t j, int64_t kc) {
+  return ((r >> 7) * kc + (j >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (j & 3);
+}
+
+// Quantize 8 elements (half a block) held by this thread; the partner lane
+// (lane ^ 1) holds the other half.  Returns the packed codes, sets *scale.
+__device__ __forceinline__ uint32_t quantize_half_block(const float (&f)[8], float g, uint32_t* scale,
+                                                        float* half_max) {
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
+  *half_max = m;
+  const float bm = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+  const float q = __fdiv_rn(bm, 6.0f);
+  const float t = __fmul_rn(q, g);
+  const uint32_t s = cvt_e4m3(t);
+  *scale = s;
+  if (s == 0) {
+    uint32_t packed = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) packed |= ((__float_as_uint(f[i]) >> 31) << 3) << (4 * i);
+    return packed;
+  }
+  const float r = __fdiv_rn(g, e4m3_to_f32(s));
+  float y[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(f[i], r);
+  return cvt_e2m1x8(y);
+}
+
+template <bool kF32>
+struct Loaded {
+  uint4 v[kF32 ? 2 : 1];
+};
+
+template <bool kF32>
+__device__ __forceinline__ void load_half(const void* x, int64_t h, Loaded<kF32>& L) {
+  if constexpr (kF32) {
+    const uint4* p = reinterpret_cast<const uint4*>(x) + 2 * h;
+    L.v[0] = __ldcs(p);
+    L.v[1] = __ldcs(p + 1);
+  } else {
+    L.v[0] = __ldcs(reinterpret_cast<const uint4*>(x) + h);
+  }
+}
+
+template <bool kF32>
+__device__ __forceinline__ void unpack(const Loaded<kF32>& L, float (&f)[8]) {
+  if constexpr (kF32) {
+    f[0] = __uint_as_float(L.v[0].x); f[1] = __uint_as_float(L.v[0].y);
+    f[2] = __uint_as_float(L.v[0].z); f[3] = __uint_as_float(L.v[0].w);
+    f[4] = __uint_as_float(L.v[1].x); f[5] = __uint_as_float(L.v[1].y);
+    f[6] = __uint_as_float(L.v[1].z); f[7] = __uint_as_float(L.v[1].w);
+  } else {
+    const uint32_t w[4] = {L.v[0].x, L.v[0].y, L.v[0].z, L.v[0].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(w[i] << 16);           // bf16 -> f32 is exact
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+}
+
+// Grid-stride over "halves" (8-element pieces).  Rows [M, rows_total) only
+// exist in the tensor-core layout (padding to 128 rows): they read nothing
+// and write zero scales.
+template <bool kF32, bool kTC, bool kAmax>
+__global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ x, int64_t M, int64_t K,
+                                                       int64_t rows_total, float g, uint8_t* __restrict__ codes,
+                                                       uint8_t* __restrict__ scales, float* amax_out,
+                                                       int64_t kc) {
+  constexpr int U = 4;
+  const int lane = threadIdx.x & 31;
+  const int64_t halves_per_row = K >> 3;
+  const int64_t total = rows_total * halves_per_row;   // even: K/8 is even
+  const int64_t real = M * halves_per_row;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t nblk = K >> 4;
+  float local_max = 0.0f;
+
+  for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < total; base += U * stride) {
+    Loaded<kF32> L[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t h = base + u * stride + lane;
+      if (h < real) load_half<kF32>(x, h, L[u]);
+      else {
+#pragma unroll
+        for (int i = 0; i < (kF32 ? 2 : 1); ++i) L[u].v[i] = make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t h = base + u * stride + lane;
+      float f[8];
+      unpack<kF32>(L[u], f);
+      uint32_t s;
+      float hm;
+      const uint32_t packed = quantize_half_block(f, g, &s, &hm);
+      local_max = fmaxf(local_max, hm);
+      if (h < real) reinterpret_cast<uint32_t*>(codes)[h] = packed;
+      if (h < total && (lane & 1) == 0) {
+        const int64_t row = h / halves_per_row;
+        const int64_t j = (h - row * halves_per_row) >> 1;
+        if constexpr (kTC) {
+          scales[tc_scale_offset(row, j, kc)] = (uint8_t)s;
+          // K % 64 == 32: the last chunk of the row has two padding slots
+          if (j == nblk - 1 && (nblk & 3) == 2) {
+            scales[tc_scale_offset(row, j + 1, kc)] = 0;
+            scales[tc_scale_offset(row, j + 2, kc)] = 0;
+          }
+        } else {
+          scales[row * nblk + j] = (uint8_t)s;
+        }
+      }
+    }
+  }
+
+  if constexpr (kAmax) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) local_max = fmaxf(local_max, __shfl_xor_sync(0xFFFFFFFFu, local_max, o));
+    __shared__ float wmax[8];
+    if (lane == 0) wmax[threadIdx.x >> 5] = local_max;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float b = 0.0f;
+      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) b = fmaxf(b, wmax[w]);
+      // non-negative floats order like their bit patterns
+      atomicMax(reinterpret_cast<unsigned*>(amax_out), __float_as_uint(b));
+    }
+  }
+}
+
+template <bool kF32>
+__global__ void __launch_bounds__(256) amax_kernel(const void* __restrict__ x, int64_t n_vec, float* amax_out) {
+  // n_vec 16-byte vectors; any tail elements are handled by the host-chosen
+  // element count being a multiple of the vector width (K*M*elt % 16 == 0).
+  float m = 0.0f;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_vec; i += stride) {
+    const uint4 v = __ldcs(reinterpret_cast<const uint4*>(x) + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if constexpr (kF32) {
+        m = fmaxf(m, fabsf(__uint_as_float(w[k])));
+      } else {
+        m = fmaxf(m, fabsf(__uint_as_float(w[k] << 16)));
+        m = fmaxf(m, fabsf(__uint_as_float(w[k] & 0xFFFF0000u)));
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  __shared__ float wmax[8];
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float b = 0.0f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) b = fmaxf(b, wmax[w]);
+    atomicMax(reinterpret_cast<unsigned*>(amax_out), __float_as_uint(b));
+  }
+}
+
+// One thread per 4-byte word of the tensor-core layout.
+__global__ void swizzle_scales_kernel(const uint8_t* __restrict__ rm, int64_t R, int64_t nblk, int64_t kc,
+                                      int64_t n_words, uint32_t* __restrict__ tc) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < n_words; w += stride) {
+    const int64_t chunk = w >> 7;
+    const int64_t o = (w & 127) * 4;
+    const int64_t rb = chunk / kc, cb = chunk - rb * kc;
+    const int64_t row = rb * 128 + (o >> 4) + 32 * ((o & 15) >> 2);
+    uint32_t word = 0;
+    if (row < R) {
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int64_t j = cb * 4 + t;
+        if (j < nblk) word |= (uint32_t)rm[row * nblk + j] << (8 * t);
+      }
+    }
+    tc[w] = word;
+  }
+}
+
+__global__ void convert_e4m3_kernel(const float* __restrict__ in, uint8_t* __restrict__ out, int64_t n) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+    out[i] = (uint8_t)cvt_e4m3(in[i]);
+}
+
+__global__ void convert_e2m1_kernel(const float* __restrict__ in, uint8_t* __restrict__ out, int64_t n_pairs) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < n_pairs; j += stride)
+    out[j] = (uint8_t)cvt_e2m1x2(in[2 * j], in[2 * j + 1]);
+}
+
+namespace {
+
+int grid_for(int64_t work_items, int threads, const DeviceInfo* d, int per_sm = 8) {
+  int64_t blocks = ceil_div(work_items, threads);
+  const int64_t cap = (int64_t)d->sm_count * per_sm;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return (int)blocks;
+}
+
+template <bool kF32, bool kTC, bool kAmax>
+cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, float g, uint8_t* codes, uint8_t* scales,
+                            float* amax_out, cudaStream_t st, const DeviceInfo* d) {
+  const int64_t rows_total = kTC ? ceil_div(M, 128) * 128 : M;
+  const int64_t kc = ceil_div(K, 64);
+  const int64_t halves = rows_total * (K / 8);
+  // each warp-iteration covers U*stride halves; size the grid so every SM
+  // holds 2048 threads when there is enough work
+  const int threads = 256;
+  int blocks = grid_for(ceil_div(halves, 4), threads, d, 8);
+  quantize_kernel<kF32, kTC, kAmax><<<blocks, threads, 0, st>>>(x, M, K, rows_total, g, codes, scales,
+                                                                amax_out, kc);
+  return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+extern "C" {
+
+size_t nvfp4_scale_bytes(int64_t rows, int64_t K, nvfp4_sf_layout layout) {
+  if (rows < 1 || K < 16 || K % 16 != 0) return 0;
+  if (layout == NVFP4_SF_ROWMAJOR) return (size_t)(rows * (K / 16));
+  if (layout == NVFP4_SF_TCGEN05) return (size_t)(ceil_div(rows, 128) * ceil_div(K, 64) * 512);
+  return 0;
+}
+
+nvfp4_status nvfp4_amax(const void* x, nvfp4_in_dtype dtype, int64_t M, int64_t K, float* amax_out,
+                        nvfp4_stream_t stream) {
+  if (!x || !amax_out || M < 1 || K < 1) return NVFP4_ERR_INVALID_ARG;
+  if (dtype != NVFP4_IN_BF16 && dtype != NVFP4_IN_F32) return NVFP4_ERR_INVALID_ARG;
+  const int64_t elt = dtype == NVFP4_IN_F32 ? 4 : 2;
+  if ((M * K * elt) % 16 != 0) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(amax_out) & 3)) return NVFP4_ERR_ALIGNMENT;
+  const DeviceInfo* d = device_info();
+  if (!d) return NVFP4_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), st);
+  if (e != cudaSuccess) return cuda_status(e);
+  const int64_t n_vec = M * K * elt / 16;
+  const int blocks = grid_for(n_vec, 256, d, 8);
+  if (dtype == NVFP4_IN_F32) amax_kernel<true><<<blocks, 256, 0, st>>>(x, n_vec, amax_out);
+  else amax_kernel<false><<<blocks, 256, 0, st>>>(x, n_vec, amax_out);
+  return cuda_status(cudaGetLastError());
+}
+
+nvfp4_status nvfp4_quantize(const void* x, nvfp4_in_dtype dtype, int64_t M, int64_t K, float global_scale,
+                            uint8_t* codes, uint8_t* block_scales, nvfp4_sf_layout layout, float* amax_out,
+                            nvfp4_stream_t stream) {
+  if (!x || !codes || !block_scales || M < 1 || K < 32 || K % 32 != 0) return NVFP4_ERR_INVALID_ARG;
+  if (dtype != NVFP4_IN_BF16 && dtype != NVFP4_IN_F32) return NVFP4_ERR_INVALID_ARG;
+  if (layout != NVFP4_SF_ROWMAJOR && layout != NVFP4_SF_TCGEN05) return NVFP4_ERR_INVALID_ARG;
+  if (!finite_positive(global_scale)) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(block_scales)) return NVFP4_ERR_ALIGNMENT;
+  if (amax_out && (reinterpret_cast<uintptr_t>(amax_out) & 3)) return NVFP4_ERR_ALIGNMENT;
+  const DeviceInfo* d = device_info();
+  if (!d) return NVFP4_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (amax_out) {
+    cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), st);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  const bool f32 = dtype == NVFP4_IN_F32, tc = layout == NVFP4_SF_TCGEN05, am = amax_out != nullptr;
+  cudaError_t e;
+#define NVFP4_Q(A, B, C) \
+  if (f32 == A && tc == B && am == C) e = launch_quantize<A, B, C>(x, M, K, global_scale, codes, block_scales, amax_out, st, d);
+  NVFP4_Q(false, false, false) else NVFP4_Q(false, false, true) else NVFP4_Q(false, true, false)
+  else NVFP4_Q(false, true, true) else NVFP4_Q(true, false, false) else NVFP4_Q(true, false, true)
+  else NVFP4_Q(true, true, false) else NVFP4_Q(true, true, true) else e = cudaErrorInvalidValue;
+#undef NVFP4_Q
+  return cuda_status(e);
+}
+
+nvfp4_status nvfp4_swizzle_scales(const uint8_t* rowmajor, int64_t rows, int64_t K, uint8_t* tc,
+                                  nvfp4_stream_t stream) {
+  if (!rowmajor || !tc || rows < 1 || K < 16 || K % 16 != 0) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(tc)) return NVFP4_ERR_ALIGNMENT;
+  const DeviceInfo* d = device_info();
+  if (!d) return NVFP4_ERR_CUDA;
+  const int64_t kc = ceil_div(K, 64);
+  const int64_t n_words = ceil_div(rows, 128) * kc * 128;
+  const int blocks = grid_for(n_words, 256, d, 8);
+  swizzle_scales_kernel<<<blocks, 256, 0, (cudaStream_t)stream>>>(rowmajor, rows, K / 16, kc, n_words,
+                                                                  reinterpret_cast<uint32_t*>(tc));
+  return cuda_status(cudaGetLastError());
+}
+
+nvfp4_status nvfp4_convert_e4m3(const float* in, uint8_t* out, int64_t n, nvfp4_stream_t stream) {
+  if (!in || !out || n < 1) return NVFP4_ERR_INVALID_ARG;
+  const DeviceInfo* d = device_info();
+  if (!d) return NVFP4_ERR_CUDA;
+  convert_e4m3_kernel<<<grid_for(n, 256, d, 8), 256, 0, (cudaStream_t)stream>>>(in, out, n);
+  return cuda_status(cudaGetLastError());
+}
+
+nvfp4_status nvfp4_convert_e2m1(const float* in, uint8_t* out, int64_t n, nvfp4_stream_t stream) {
+  if (!in || !out || n < 2 || (n & 1)) return NVFP4_ERR_INVALID_ARG;
+  const DeviceInfo* d = device_info();
+  if (!d) return NVFP4_ERR_CUDA;
+  convert_e2m1_kernel<<<grid_for(n / 2, 256, d, 8), 256, 0, (cudaStream_t)stream>>>(in, out, n / 2);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // extern "C"
