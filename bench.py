@@ -75,6 +75,14 @@ def profiled_traffic(kernel: str, workload: str):
 
 # ----------------------------------------------------------------- clocks
 
+def smi_id(props, index: int) -> str:
+    """nvidia-smi --id for a torch device: its PCI address when known."""
+    try:
+        return f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+    except Exception:
+        return str(index)
+
+
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -382,73 +390,29 @@ def run_reference(args):
     return 0
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-extra", action="store_true")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    args = ap.parse_args()
-    args.warmup = max(3, args.warmup)
-    if args.impl == "reference":
-        return run_reference(args)
-
-    import torch
-    import nvfp4_w4a4_quantized_10_b200 as nv
-    import synth
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    pg = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-        pg = dist
-
-    def barrier():
-        if pg is not None:
-            pg.barrier()
-        torch.cuda.synchronize()
-
-    def max_over_ranks(v: float) -> float:
-        return aggregate_replicas(v, 0.0, world, pg, dev)[0]
-
-    peaks, peak_kind = load_peaks()
-    props = torch.cuda.get_device_properties(dev)
-    l2 = getattr(props, "L2_cache_size", 126 * 1024 * 1024) or 126 * 1024 * 1024
-    sampler = ClockSampler(local)
-    sampler.start()
-    stream = torch.cuda.Stream(device=dev)
-
-    # ---- headline: decode step
+def measure_decode(torch, nv, synth, dev, rank, world, l2, args, stream, barrier, max_over_ranks, peaks,
+                   peak_kind):
     d = Decode(torch, nv, synth, dev, rank, l2)
     torch.cuda.synchronize()
-    # soak so the clock sampler sees the GPU under this load
+    # soak so the clock sampler sees the GPU under this load before timing
     t_soak = time.time()
     i = 0
-    while time.time() - t_soak < 1.0:
+    while time.time() - t_soak < args.soak:
         d.step(i)
         i += 1
         if i % 64 == 0:
             torch.cuda.synchronize()
     barrier()
-    t0 = time.time()
     with torch.cuda.stream(stream):
         ms_step, g_step = time_graph(torch, d.step, args.steps, args.warmup, stream)
         ms_gemm, g_gemm = time_graph(torch, d.gemm_only, args.steps, args.warmup, stream)
     barrier()
-    t1 = time.time()
+    t_end = time.time()
     ms_step = max_over_ranks(ms_step)
     ms_gemm = max_over_ranks(ms_gemm)
     del g_step, g_gemm
 
-    # ---- end to end through the public API: pinned host X in, host result out
+    # end to end through the public API: pinned host X in, host result out
     x_host = d.x.cpu().pin_memory()
     out_host = torch.empty(d.out.shape, dtype=d.out.dtype).pin_memory()
     x_dev = torch.empty_like(d.x)
@@ -483,58 +447,139 @@ def main():
                 "d2h_bytes_per_step": d.out.numel() * d.out.element_size()},
         "gpu_launches": d.launches_per_step * args.steps,
     }
-    clk = sampler.summary(t_soak, t1)
     del d
+    return line, t_soak, t_end
 
-    # ---- extra workloads (rank 0 measures them only at N = 1)
+
+def measure_prefill(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind):
+    w = synth.PREFILL
+    if args.prefill_m:
+        import dataclasses
+        w = dataclasses.replace(w, M=args.prefill_m)
+    p = Prefill(torch, nv, synth, dev, rank, l2, w)
+    k = max(3, min(args.steps, 20))
+    with torch.cuda.stream(stream):
+        ms_p, g1 = time_graph(torch, p.step, k, 3, stream)
+        ms_pg, g2 = time_graph(torch, p.gemm_only, k, 3, stream)
+    del g1, g2
+    fp4_peak = float(peaks["bf16_tflops"]) * FP4_OVER_BF16
+    fp4_sust = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])) * FP4_OVER_BF16
+    tf = p.flops / (ms_pg * 1e-3) / 1e12
+    res = {
+        "workload": f"prefill-shape linear X[{w.M},5120] bf16 x W[17408,5120] nvfp4 -> bf16",
+        "step_tflops": p.flops / (ms_p * 1e-3) / 1e12, "ms_per_step": ms_p,
+        "roofline": {"bound": "tensor", "kernel": "nvfp4_gemm_kernel<256>", "achieved": tf,
+                     "peak": fp4_peak, "unit": "TFLOP/s", "frac": tf / fp4_peak,
+                     "frac_of_sustained": tf / fp4_sust,
+                     "peak_kind": f"{peak_kind} bf16 cuBLAS x {FP4_OVER_BF16:g} (nominal fp4/bf16)",
+                     "flops_per_launch": p.flops, "ms_per_launch": ms_pg,
+                     "traffic": profiled_traffic("nvfp4_gemm_kernel", "prefill")},
+        "l2": "inputs 129 MB + 1.14 GB output per step exceed L2"}
+    del p
+    return res
+
+
+def measure_fused(torch, nv, synth, dev, rank, l2, args, stream):
+    f = FusedGDN(torch, nv, synth, dev, rank, l2)
+    k = max(3, min(args.steps, 20))
+    with torch.cuda.stream(stream):
+        ms_f, g3 = time_graph(torch, f.step, k, 3, stream)
+    del g3
+    res = {"workload": "fused GDN projection X[4096,5120] x W[8192|4096|48|48, 5120]",
+           "step_tflops": f.flops / (ms_f * 1e-3) / 1e12, "ms_per_step": ms_f}
+    del f
+    return res
+
+
+def measure_quant_sweep(torch, nv, synth, dev, args, stream, peaks):
+    hbm_peak = float(peaks["hbm_gbs"])
+    sweep = {}
+    for M in synth.QUANT_SWEEP_M:
+        for K in synth.QUANT_SWEEP_K:
+            q = QuantSweep(torch, nv, synth, dev, M, K)
+            kk = max(3, min(args.steps, 50))
+            with torch.cuda.stream(stream):
+                ms_q, g4 = time_graph(torch, q.step, kk, 3, stream)
+            del g4
+            gbs = q.bytes / (ms_q * 1e-3) / 1e9
+            sweep[f"{M}x{K}"] = {"us": ms_q * 1e3, "GB/s": gbs, "frac_hbm": gbs / hbm_peak}
+            del q
+    return sweep
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--only", default="all", choices=["all", "decode", "prefill", "fused", "quant"])
+    ap.add_argument("--prefill-m", type=int, default=0, help="override M of the prefill workload")
+    ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed decode steps first")
+    ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import nvfp4_w4a4_quantized_10_b200 as nv
+    import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(v: float) -> float:
+        return aggregate_replicas(v, 0.0, world, pg, dev)[0]
+
+    peaks, peak_kind = load_peaks()
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 126 * 1024 * 1024) or 126 * 1024 * 1024
+    sampler = ClockSampler(smi_id(props, local))
+    sampler.start()
+    stream = torch.cuda.Stream(device=dev)
+
+    if args.only != "all" and world == 1:
+        if args.only == "decode":
+            res, _, _ = measure_decode(torch, nv, synth, dev, rank, world, l2, args, stream, barrier,
+                                       max_over_ranks, peaks, peak_kind)
+        elif args.only == "prefill":
+            res = measure_prefill(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind)
+        elif args.only == "fused":
+            res = measure_fused(torch, nv, synth, dev, rank, l2, args, stream)
+        else:
+            res = measure_quant_sweep(torch, nv, synth, dev, args, stream, peaks)
+        sampler.stop()
+        print(json.dumps({"only": args.only, "result": res}))
+        return 0
+
+    line, t_soak, t_end = measure_decode(torch, nv, synth, dev, rank, world, l2, args, stream, barrier,
+                                         max_over_ranks, peaks, peak_kind)
+    clk = sampler.summary(t_soak, t_end)
     if not args.no_extra and world == 1:
-        extra = {}
-        p = Prefill(torch, nv, synth, dev, rank, l2)
-        k = max(3, min(args.steps, 20))
-        with torch.cuda.stream(stream):
-            ms_p, g1 = time_graph(torch, p.step, k, 3, stream)
-            ms_pg, g2 = time_graph(torch, p.gemm_only, k, 3, stream)
-        del g1, g2
-        fp4_peak = float(peaks["bf16_tflops"]) * FP4_OVER_BF16
-        fp4_sust = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])) * FP4_OVER_BF16
-        tf = p.flops / (ms_pg * 1e-3) / 1e12
-        extra["prefill"] = {
-            "workload": "prefill-shape linear X[32768,5120] bf16 x W[17408,5120] nvfp4 -> bf16",
-            "step_tflops": p.flops / (ms_p * 1e-3) / 1e12, "ms_per_step": ms_p,
-            "roofline": {"bound": "tensor", "kernel": "nvfp4_gemm_kernel<256>", "achieved": tf,
-                         "peak": fp4_peak, "unit": "TFLOP/s", "frac": tf / fp4_peak,
-                         "frac_of_sustained": tf / fp4_sust,
-                         "peak_kind": f"{peak_kind} bf16 cuBLAS x {FP4_OVER_BF16:g} (nominal fp4/bf16)",
-                         "flops_per_launch": p.flops, "ms_per_launch": ms_pg,
-                         "traffic": profiled_traffic("nvfp4_gemm_kernel", "prefill")},
-            "l2": "inputs 129 MB + 1.14 GB output per step exceed L2"}
-        del p
-        f = FusedGDN(torch, nv, synth, dev, rank, l2)
-        with torch.cuda.stream(stream):
-            ms_f, g3 = time_graph(torch, f.step, k, 3, stream)
-        del g3
-        extra["fused_gdn"] = {"workload": "fused GDN projection X[4096,5120] x W[8192|4096|48|48, 5120]",
-                              "step_tflops": f.flops / (ms_f * 1e-3) / 1e12, "ms_per_step": ms_f}
-        del f
-        sweep = {}
-        for M in synth.QUANT_SWEEP_M:
-            for K in synth.QUANT_SWEEP_K:
-                q = QuantSweep(torch, nv, synth, dev, M, K)
-                kk = max(3, min(args.steps, 50))
-                # rotate nothing: M >= 4096 tensors exceed L2 together with their outputs
-                with torch.cuda.stream(stream):
-                    ms_q, g4 = time_graph(torch, q.step, kk, 3, stream)
-                del g4
-                sweep[f"{M}x{K}"] = {"us": ms_q * 1e3, "GB/s": q.bytes / (ms_q * 1e-3) / 1e9,
-                                     "frac_hbm": q.bytes / (ms_q * 1e-3) / 1e9 / hbm_peak}
-                del q
-        extra["quantize_sweep"] = sweep
-        line["extra"] = extra
-
+        line["extra"] = {
+            "prefill": measure_prefill(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind),
+            "fused_gdn": measure_fused(torch, nv, synth, dev, rank, l2, args, stream),
+            "quantize_sweep": measure_quant_sweep(torch, nv, synth, dev, args, stream, peaks),
+        }
     sampler.stop()
     if clk is not None:
         line["clocks"] = clk
-
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu, _, _ = oracle_decode_sample()
         line["cpu_baseline"] = cpu
