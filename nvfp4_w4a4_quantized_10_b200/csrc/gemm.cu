@@ -48,10 +48,13 @@ constexpr int kSfChunk = 512;     // bytes of one 128-row x 4-scale chunk
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
 constexpr int kGroupP = 8;        // tile raster: 8 P-tiles share a Q-tile
+constexpr int kStageOutBytes = 16384;   // one 128-row x 128-byte output sub-tile
+constexpr int kEpiBar = 1;        // named barrier id of the 128 epilogue threads
 
 struct alignas(64) GemmParams {
   CUtensorMap tmap_p;
   CUtensorMap tmap_q;
+  CUtensorMap tmap_out;  // output [M, N] in 128-byte-wide boxes (normal tiles, TMA store path)
   const uint8_t* sf_p;
   const uint8_t* sf_q;
   void* out;
@@ -63,6 +66,7 @@ struct alignas(64) GemmParams {
   int kc;                // ceil(K / 64): scale chunks per row block
   int kt;                // ceil(K / 256): pipeline steps per tile
   int tiles_p, tiles_q;
+  int tma_store;         // 1: output through shared memory and TMA stores
   int n_seg;
   int seg_end[NVFP4_MAX_SEGMENTS];
   float seg_alpha[NVFP4_MAX_SEGMENTS];
@@ -76,34 +80,30 @@ struct Cfg {
   static constexpr int kSfaBytes = 4 * kSfChunk;                     // 2 KB
   static constexpr int kSfbBytes = kSfbBlocks * 4 * kSfChunk;
   static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  static constexpr int kOutBytes = SWAP ? 0 : 2 * kStageOutBytes;    // double-buffered output sub-tiles
   static constexpr int kMaxStages = SWAP ? 8 : 4;
-  static constexpr int kStages =
-      (220 * 1024) / kStageBytes < kMaxStages ? (220 * 1024) / kStageBytes : kMaxStages;
+  static constexpr int kFit = (222 * 1024 - kOutBytes) / kStageBytes;
+  static constexpr int kStages = kFit < kMaxStages ? kFit : kMaxStages;
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + kStages * kABytes;
   static constexpr int kOffSfa = kOffB + kStages * kBBytes;
   static constexpr int kOffSfb = kOffSfa + kStages * kSfaBytes;
-  static constexpr int kOffBar = kOffSfb + kStages * kSfbBytes;
+  static constexpr int kOffOut = kOffSfb + kStages * kSfbBytes;      // 1024-aligned
+  static constexpr int kOffBar = kOffOut + kOutBytes;
   static constexpr int kNumBars = 2 * kStages + 3;                   // full, empty, acc_full, acc_empty, drain
-  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kOffSeg = kOffBar + kNumBars * 8;             // segment table: ends, alphas
+  static constexpr int kOffMisc = kOffSeg + 2 * 4 * NVFP4_MAX_SEGMENTS;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;            // + alignment slack
   // TMEM columns: accumulator, then per-stage scale regions
   static constexpr int kAccCols = BN < 32 ? 32 : BN;
   static constexpr int kSfaCols = 16;                                // 4 MMAs x 4 columns
   static constexpr int kSfbCols = kSfbBlocks * 16;
   static constexpr int kSfStageCols = kSfaCols + kSfbCols;
+  static_assert(kStages >= 2, "pipeline depth");
   static_assert(kAccCols + kStages * kSfStageCols <= kTmemCols, "TMEM budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(BN % 16 == 0 && BN <= 256, "MMA N");
 };
-
-__device__ __forceinline__ int seg_index(const GemmParams& p, int64_t n) {
-  int i = 0;
-  while (i < p.n_seg - 1 && n >= p.seg_end[i]) ++i;
-  return i;
-}
-
-__device__ __forceinline__ float seg_alpha(const GemmParams& p, int64_t n) { return p.seg_alpha[seg_index(p, n)]; }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);   // round to nearest even
@@ -120,6 +120,21 @@ __device__ __forceinline__ void tile_coords(const GemmParams& p, int tile, int& 
   tq = local / gsize;
 }
 
+// Segment of output column n, from the table the CTA copied to shared memory.
+__device__ __forceinline__ int seg_index_smem(const int* ends, int n_seg, int64_t n) {
+  int i = 0;
+  while (i < n_seg - 1 && n >= ends[i]) ++i;
+  return i;
+}
+
+__device__ __forceinline__ float seg_alpha_smem(const int* ends, const float* alphas, int n_seg, int64_t n) {
+  return alphas[seg_index_smem(ends, n_seg, n)];
+}
+
+// Byte offset of 16-byte chunk c of row r in a 128-row x 128-byte sub-tile
+// stored with the 128B swizzle the output tensor map uses.
+__device__ __forceinline__ uint32_t swz128(uint32_t r, uint32_t c) { return r * 128 + ((c ^ (r & 7)) << 4); }
+
 template <int BN, bool SWAP, bool OUT_F32>
 __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_constant__ GemmParams p) {
   using C = Cfg<BN, SWAP>;
@@ -131,6 +146,8 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
   const uint32_t bar_acc_full = bar_empty + 8 * C::kStages;
   const uint32_t bar_acc_empty = bar_acc_full + 8;
   const uint32_t bar_drain = bar_acc_empty + 8;
+  int* seg_end_s = reinterpret_cast<int*>(smem + C::kOffSeg);
+  float* seg_alpha_s = reinterpret_cast<float*>(smem + C::kOffSeg + 4 * NVFP4_MAX_SEGMENTS);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -150,6 +167,11 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
     fence_barrier_init();
     prefetch_tmap(&p.tmap_p);
     prefetch_tmap(&p.tmap_q);
+    if (!SWAP && p.tma_store) prefetch_tmap(&p.tmap_out);
+  }
+  if (threadIdx.x >= 64 && threadIdx.x < 64 + NVFP4_MAX_SEGMENTS) {
+    seg_end_s[threadIdx.x - 64] = p.seg_end[threadIdx.x - 64];
+    seg_alpha_s[threadIdx.x - 64] = p.seg_alpha[threadIdx.x - 64];
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), kTmemCols);
@@ -167,31 +189,31 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
       uint32_t phase = 0;
       uint32_t issued_mask = 0, last_parity = 0;   // for the drain on abort
       bool ok = true;
+      const int kt = p.kt, kc = p.kc, rb_q = p.rb_q;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
         int tp, tq;
         tile_coords(p, tile, tp, tq);
         const int p0 = tp * kBM, q0 = tq * BN;
-        const uint8_t* sfp = p.sf_p + (size_t)(p0 >> 7) * p.kc * kSfChunk;
-        for (int k = 0; k < p.kt; ++k) {
-          if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, p.err, p.timeout_ns)) { ok = false; break; }
-          const int nch = min(4, p.kc - 4 * k);
-          const uint32_t sf_bytes = (uint32_t)nch * kSfChunk;
-          int nsfb = 0;
+        const uint8_t* sfp = p.sf_p + (size_t)(p0 >> 7) * kc * kSfChunk;
+        const uint8_t* sfq = p.sf_q + (size_t)(q0 >> 7) * kc * kSfChunk;
+        int nsfb = 0;
 #pragma unroll
-          for (int rb = 0; rb < C::kSfbBlocks; ++rb)
-            if ((q0 >> 7) + rb < p.rb_q) ++nsfb;
+        for (int rb = 0; rb < C::kSfbBlocks; ++rb)
+          if ((q0 >> 7) + rb < rb_q) ++nsfb;
+        for (int k = 0; k < kt; ++k) {
+          if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, p.err, p.timeout_ns)) { ok = false; break; }
+          const int nch = min(4, kc - 4 * k);
+          const uint32_t sf_bytes = (uint32_t)nch * kSfChunk;
           const uint32_t fb = bar_full + 8 * stage;
           mbar_arrive_expect_tx(fb, C::kABytes + C::kBBytes + sf_bytes * (1 + nsfb));
           tma_load_2d(sbase + C::kOffA + stage * C::kABytes, &p.tmap_p, k * kBKBytes, p0, fb);
           tma_load_2d(sbase + C::kOffB + stage * C::kBBytes, &p.tmap_q, k * kBKBytes, q0, fb);
           bulk_load(sbase + C::kOffSfa + stage * C::kSfaBytes, sfp + (size_t)(4 * k) * kSfChunk, sf_bytes, fb);
 #pragma unroll
-          for (int rb = 0; rb < C::kSfbBlocks; ++rb) {
-            const int qb = (q0 >> 7) + rb;
-            if (qb < p.rb_q)
+          for (int rb = 0; rb < C::kSfbBlocks; ++rb)
+            if (rb < nsfb)
               bulk_load(sbase + C::kOffSfb + stage * C::kSfbBytes + rb * 4 * kSfChunk,
-                        p.sf_q + ((size_t)qb * p.kc + 4 * k) * kSfChunk, sf_bytes, fb);
-          }
+                        sfq + ((size_t)rb * kc + 4 * k) * kSfChunk, sf_bytes, fb);
           issued_mask |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
@@ -210,38 +232,56 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_nvf4(kBM, BN);
+      // Descriptors of stage 0, k-block 0; later stages and k-blocks only move
+      // the 14-bit start-address field (address >> 4), which never carries.
+      const uint64_t a_desc0 = smem_desc(sbase + C::kOffA, 16, 1024, 2);
+      const uint64_t b_desc0 = smem_desc(sbase + C::kOffB, 16, 1024, 2);
+      const uint64_t sfa_desc0 = smem_desc(sbase + C::kOffSfa, 16, 128, 0);
+      const uint64_t sfb_desc0 = smem_desc(sbase + C::kOffSfb, 16, 128, 0);
       const uint32_t acc = tmem_base;
+      const uint32_t sf_t0 = tmem_base + C::kAccCols;
+      const int kt = p.kt, kc = p.kc;
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
         if (!mbar_wait(bar_acc_empty, acc_phase ^ 1, abort_flag, p.err, p.timeout_ns)) break;
         tc_fence_after();
-        for (int k = 0; k < p.kt; ++k) {
+        for (int k = 0; k < kt; ++k) {
           if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, p.err, p.timeout_ns)) { ok = false; break; }
           tc_fence_after();
-          const int nkb = min(4, p.kc - 4 * k);
-          const uint32_t sfa_t = tmem_base + C::kAccCols + stage * C::kSfStageCols;
+          const uint32_t sfa_t = sf_t0 + stage * C::kSfStageCols;
           const uint32_t sfb_t = sfa_t + C::kSfaCols;
-          const uint32_t sa = sbase + C::kOffSfa + stage * C::kSfaBytes;
-          const uint32_t sb = sbase + C::kOffSfb + stage * C::kSfbBytes;
-          for (int kb = 0; kb < nkb; ++kb) {
-            // 32 rows x 16 bytes, core matrices of 8 rows 128 bytes apart
-            tc_cp_32x128b_warpx4(sfa_t + kb * 4, smem_desc(sa + kb * kSfChunk, 16, 128, 0));
+          const uint64_t ad = a_desc0 + (uint64_t)((stage * C::kABytes) >> 4);
+          const uint64_t bd = b_desc0 + (uint64_t)((stage * C::kBBytes) >> 4);
+          const uint64_t sad = sfa_desc0 + (uint64_t)((stage * C::kSfaBytes) >> 4);
+          const uint64_t sbd = sfb_desc0 + (uint64_t)((stage * C::kSfbBytes) >> 4);
+          const uint32_t acc_in = k != 0 ? 1u : 0u;
+          if (4 * k + 4 <= kc) {
 #pragma unroll
-            for (int rb = 0; rb < C::kSfbBlocks; ++rb)
-              tc_cp_32x128b_warpx4(sfb_t + kb * 4 * C::kSfbBlocks + rb * 4,
-                                   smem_desc(sb + rb * 4 * kSfChunk + kb * kSfChunk, 16, 128, 0));
-          }
-          const uint32_t a_s = sbase + C::kOffA + stage * C::kABytes;
-          const uint32_t b_s = sbase + C::kOffB + stage * C::kBBytes;
-          for (int kb = 0; kb < nkb; ++kb) {
-            // K-major, 128B swizzle: 8-row groups 1024 bytes apart; a K step
-            // of 64 FP4 elements is 32 bytes inside the swizzle atom
-            const uint64_t ad = smem_desc(a_s + kb * 32, 16, 1024, 2);
-            const uint64_t bd = smem_desc(b_s + kb * 32, 16, 1024, 2);
-            tc_mma_nvf4(acc, ad, bd, idesc, sfa_t + kb * 4, sfb_t + kb * 4 * C::kSfbBlocks,
-                        (k | kb) != 0 ? 1u : 0u);
+            for (int kb = 0; kb < 4; ++kb) {
+              tc_cp_32x128b_warpx4(sfa_t + kb * 4, sad + (uint64_t)(kb * (kSfChunk >> 4)));
+#pragma unroll
+              for (int rb = 0; rb < C::kSfbBlocks; ++rb)
+                tc_cp_32x128b_warpx4(sfb_t + kb * 4 * C::kSfbBlocks + rb * 4,
+                                     sbd + (uint64_t)((rb * 4 + kb) * (kSfChunk >> 4)));
+            }
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb)
+              tc_mma_nvf4(acc, ad + (uint64_t)(kb * 2), bd + (uint64_t)(kb * 2), idesc, sfa_t + kb * 4,
+                          sfb_t + kb * 4 * C::kSfbBlocks, (acc_in | kb) != 0 ? 1u : 0u);
+          } else {
+            const int nkb = kc - 4 * k;
+            for (int kb = 0; kb < nkb; ++kb) {
+              tc_cp_32x128b_warpx4(sfa_t + kb * 4, sad + (uint64_t)(kb * (kSfChunk >> 4)));
+#pragma unroll
+              for (int rb = 0; rb < C::kSfbBlocks; ++rb)
+                tc_cp_32x128b_warpx4(sfb_t + kb * 4 * C::kSfbBlocks + rb * 4,
+                                     sbd + (uint64_t)((rb * 4 + kb) * (kSfChunk >> 4)));
+            }
+            for (int kb = 0; kb < nkb; ++kb)
+              tc_mma_nvf4(acc, ad + (uint64_t)(kb * 2), bd + (uint64_t)(kb * 2), idesc, sfa_t + kb * 4,
+                          sfb_t + kb * 4 * C::kSfbBlocks, (acc_in | kb) != 0 ? 1u : 0u);
           }
           tc_commit(bar_empty + 8 * stage);
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
@@ -260,8 +300,14 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
     // ------------------------------------------------------------ epilogue
     const int sp = warp & 3;                 // TMEM subpartition of this warp
     const int row = sp * 32 + lane;          // accumulator lane = tile row of P
+    const int et = threadIdx.x - 64;         // epilogue thread index 0..127
     const uint32_t taddr = tmem_base + ((uint32_t)(sp * 32) << 16);
+    const int64_t M = p.M, N = p.N;
+    const int n_seg = p.n_seg;
+    const float alpha0 = seg_alpha_s[0];
+    const bool tma_store = !SWAP && p.tma_store;
     uint32_t acc_phase = 0;
+    uint32_t out_buf = 0;                    // next staging buffer (TMA store path)
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
       int tp, tq;
       tile_coords(p, tile, tp, tq);
@@ -272,56 +318,108 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
       if constexpr (!SWAP) {
         const int64_t m = p0 + row;
         if constexpr (!OUT_F32) {
+          // drain the whole accumulator row into registers (bf16 pairs), then
+          // hand TMEM back to the MMA warp before any store
           uint32_t packed[BN / 2];
 #pragma unroll
-          for (int c = 0; c < BN / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(taddr + c * 32, r);
+          for (int c = 0; c < BN / 32; c += 2) {
+            uint32_t r0[32], r1[32];
+            tmem_ld_32x32b_x32(taddr + c * 32, r0);
+            tmem_ld_32x32b_x32(taddr + (c + 1) * 32, r1);
             tmem_ld_wait();
-            const int64_t nb = q0 + c * 32;
-            const bool uniform = seg_index(p, nb) == seg_index(p, nb + 31);
-            const float a0 = seg_alpha(p, nb);
+            float a[2] = {alpha0, alpha0};
+            const bool seg_uniform =
+                n_seg == 1 || seg_index_smem(seg_end_s, n_seg, q0 + c * 32) ==
+                                  seg_index_smem(seg_end_s, n_seg, q0 + c * 32 + 63);
+            if (seg_uniform) a[0] = a[1] = seg_alpha_smem(seg_end_s, seg_alpha_s, n_seg, q0 + c * 32);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float alo = uniform ? a0 : seg_alpha(p, nb + 2 * i);
-              const float ahi = uniform ? a0 : seg_alpha(p, nb + 2 * i + 1);
-              packed[c * 16 + i] = pack_bf16x2(__fmul_rn(__uint_as_float(r[2 * i]), alo),
-                                               __fmul_rn(__uint_as_float(r[2 * i + 1]), ahi));
+              float alo = a[0], ahi = a[0], blo = a[1], bhi = a[1];
+              if (!seg_uniform) {
+                alo = seg_alpha_smem(seg_end_s, seg_alpha_s, n_seg, q0 + c * 32 + 2 * i);
+                ahi = seg_alpha_smem(seg_end_s, seg_alpha_s, n_seg, q0 + c * 32 + 2 * i + 1);
+                blo = seg_alpha_smem(seg_end_s, seg_alpha_s, n_seg, q0 + c * 32 + 32 + 2 * i);
+                bhi = seg_alpha_smem(seg_end_s, seg_alpha_s, n_seg, q0 + c * 32 + 33 + 2 * i);
+              }
+              packed[c * 16 + i] = pack_bf16x2(__fmul_rn(__uint_as_float(r0[2 * i]), alo),
+                                               __fmul_rn(__uint_as_float(r0[2 * i + 1]), ahi));
+              packed[(c + 1) * 16 + i] = pack_bf16x2(__fmul_rn(__uint_as_float(r1[2 * i]), blo),
+                                                     __fmul_rn(__uint_as_float(r1[2 * i + 1]), bhi));
             }
           }
           tc_fence_before();
           mbar_arrive(bar_acc_empty);
-          if (m < p.M) {
-            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + m * p.N;
-            const bool vec = (p.N % 8) == 0;
+          if (tma_store) {
+            // 64-column sub-tiles through two 16 KB swizzled staging buffers
+#pragma unroll
+            for (int sub = 0; sub < BN / 64; ++sub) {
+              // sub-tiles wholly past N are skipped outright (uniform across
+              // the epilogue), so every buffer written is one whose last
+              // store has been committed and waited for
+              if (q0 + sub * 64 >= N) continue;
+              const uint32_t buf = sbase + C::kOffOut + out_buf * kStageOutBytes;
+              if (et == 0) bulk_wait_group_read<1>();          // the store that used buf has read it
+              named_bar_sync(kEpiBar, 128);
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                const uint32_t* v = &packed[sub * 32 + c * 4];
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(buf + swz128(row, c)), "r"(v[0]),
+                             "r"(v[1]), "r"(v[2]), "r"(v[3])
+                             : "memory");
+              }
+              fence_proxy_async_smem();
+              named_bar_sync(kEpiBar, 128);
+              if (et == 0) {
+                tma_store_2d(&p.tmap_out, buf, (int32_t)(q0 + sub * 64), (int32_t)p0);
+                bulk_commit_group();
+              }
+              out_buf ^= 1;
+            }
+          } else if (m < M) {
+            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + m * N;
 #pragma unroll
             for (int c = 0; c < BN / 8; ++c) {
               const int64_t n = q0 + c * 8;
-              if (vec && n + 8 <= p.N) {
-                *reinterpret_cast<uint4*>(orow + n) =
-                    make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
-              } else {
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                  if (n + e < p.N)
-                    reinterpret_cast<uint16_t*>(orow)[n + e] =
-                        (uint16_t)(packed[4 * c + e / 2] >> (16 * (e & 1)));
-              }
+              for (int e = 0; e < 8; ++e)
+                if (n + e < N)
+                  reinterpret_cast<uint16_t*>(orow)[n + e] = (uint16_t)(packed[4 * c + e / 2] >> (16 * (e & 1)));
             }
           }
         } else {
-          float* orow = reinterpret_cast<float*>(p.out) + m * p.N;
+          // FP32 output: 32-column chunks; TMEM is released after the last one
 #pragma unroll 1
           for (int c = 0; c < BN / 32; ++c) {
             uint32_t r[32];
             __syncwarp();
             tmem_ld_32x32b_x32(taddr + c * 32, r);
             tmem_ld_wait();
-            if (m < p.M) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              r[i] = __float_as_uint(
+                  __fmul_rn(__uint_as_float(r[i]), seg_alpha_smem(seg_end_s, seg_alpha_s, n_seg, q0 + c * 32 + i)));
+            if (tma_store && q0 + c * 32 < N) {
+              const uint32_t buf = sbase + C::kOffOut + out_buf * kStageOutBytes;
+              if (et == 0) bulk_wait_group_read<1>();
+              named_bar_sync(kEpiBar, 128);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(buf + swz128(row, j)),
+                             "r"(r[4 * j]), "r"(r[4 * j + 1]), "r"(r[4 * j + 2]), "r"(r[4 * j + 3])
+                             : "memory");
+              fence_proxy_async_smem();
+              named_bar_sync(kEpiBar, 128);
+              if (et == 0) {
+                tma_store_2d(&p.tmap_out, buf, (int32_t)(q0 + c * 32), (int32_t)p0);
+                bulk_commit_group();
+              }
+              out_buf ^= 1;
+            } else if (!tma_store && m < M) {
+              float* orow = reinterpret_cast<float*>(p.out) + m * N;
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
                 const int64_t n = q0 + c * 32 + i;
-                if (n < p.N) orow[n] = __fmul_rn(__uint_as_float(r[i]), seg_alpha(p, n));
+                if (n < N) orow[n] = __uint_as_float(r[i]);
               }
             }
           }
@@ -331,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
       } else {
         // swap: lane = weight row = output column n; accumulator column = activation row
         const int64_t n = p0 + row;
-        const float alpha = seg_alpha(p, n);
+        const float alpha = seg_alpha_smem(seg_end_s, seg_alpha_s, n_seg, n);
 #pragma unroll
         for (int c = 0; c < (BN + 31) / 32; ++c) {
           uint32_t r[32];
@@ -348,14 +446,14 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
             }
           }
           tmem_ld_wait();
-          if (n < p.N) {
+          if (n < N) {
 #pragma unroll
             for (int i = 0; i < (BN < 32 ? BN : 32); ++i) {
-              const int64_t m = q0 + c * 32 + i;
-              if (m < p.M) {
+              const int64_t mm = q0 + c * 32 + i;
+              if (mm < M) {
                 const float v = __fmul_rn(__uint_as_float(r[i]), alpha);
-                if constexpr (OUT_F32) reinterpret_cast<float*>(p.out)[m * p.N + n] = v;
-                else reinterpret_cast<__nv_bfloat16*>(p.out)[m * p.N + n] = __float2bfloat16_rn(v);
+                if constexpr (OUT_F32) reinterpret_cast<float*>(p.out)[mm * N + n] = v;
+                else reinterpret_cast<__nv_bfloat16*>(p.out)[mm * N + n] = __float2bfloat16_rn(v);
               }
             }
           }
@@ -365,6 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
       }
       acc_phase ^= 1;
     }
+    if (tma_store && et == 0) bulk_wait_group<0>();   // stores done before the CTA's smem goes away
   }
 
   tc_fence_before();
@@ -409,6 +508,20 @@ bool make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, in
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Output [M, N] (bf16 or f32), boxes of 128 rows x 128 bytes, 128B swizzle.
+bool make_out_map(CUtensorMap* m, void* base, int64_t M, int64_t N, bool f32) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const int64_t esz = f32 ? 4 : 2;
+  const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+  const cuuint64_t strides[1] = {(cuuint64_t)(N * esz)};
+  const cuuint32_t box[2] = {(cuuint32_t)(128 / esz), (cuuint32_t)kBM};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -463,6 +576,10 @@ nvfp4_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float ga,
   if (!make_code_map(&p.tmap_p, codes_p, p.rows_p, K, kBM) || !make_code_map(&p.tmap_q, codes_q, p.rows_q, K, bn))
     return NVFP4_ERR_CUDA;
   p.out = out;
+  // TMA stores need 16-byte aligned output rows
+  const bool f32 = out_dtype == NVFP4_OUT_F32;
+  p.tma_store = (!swap && (N * (f32 ? 4 : 2)) % 16 == 0) ? 1 : 0;
+  if (p.tma_store && !make_out_map(&p.tmap_out, out, M, N, f32)) return NVFP4_ERR_CUDA;
   p.err = d->err_word;
   p.timeout_ns = wait_timeout_ns();
   p.M = M;
@@ -477,7 +594,6 @@ nvfp4_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float ga,
     p.seg_end[i] = (int)seg_offsets[i + 1];
     p.seg_alpha[i] = alpha_of(ga, seg_gs[i]);
   }
-  const bool f32 = out_dtype == NVFP4_OUT_F32;
   cudaError_t e;
   if (!swap) e = f32 ? launch<256, false, true>(p, d, st) : launch<256, false, false>(p, d, st);
   else if (bn == 16) e = f32 ? launch<16, true, true>(p, d, st) : launch<16, true, false>(p, d, st);

@@ -9,12 +9,12 @@
 // All FP32 steps use explicitly rounded intrinsics (no contraction), and the
 // FP8/FP4 encodings use the hardware cvt.rn.satfinite conversions.
 //
-// Work split: two adjacent threads own one 16-element block (8 elements, one
-// 16-byte bf16 load each), exchange their half maxima with one shuffle, and
-// each writes 4 bytes of codes, so a warp reads 512 contiguous bytes and
-// writes 128 contiguous bytes.  The kernel is HBM-bound (2.5625 bytes per
-// bf16 element); four independent loads per thread are in flight per
-// iteration.
+// Work split: one thread owns one 16-element block (two 16-byte loads for
+// bf16), so the per-block scalar work (two FP32 roundings, the E4M3
+// conversion, the scale store) is done once per 16 elements; a warp reads
+// 1 KB and writes 256 contiguous bytes of codes.  The kernel is meant to be
+// HBM-bound (2.5625 bytes per bf16 element); each thread keeps two blocks
+// (four 16-byte loads) in flight per iteration.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -68,131 +68,176 @@ __device__ __forceinline__ int64_t tc_scale_offset(int64_t r, int64_t j, int64_t
   return ((r >> 7) * kc + (j >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (j & 3);
 }
 
-// Quantize 8 elements (half a block) held by this thread; the partner lane
-// (lane ^ 1) holds the other half.  Returns the packed codes, sets *scale.
-__device__ __forceinline__ uint32_t quantize_half_block(const float (&f)[8], float g, uint32_t* scale,
-                                                        float* half_max) {
-  float m = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
-  *half_max = m;
-  const float bm = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-  const float q = __fdiv_rn(bm, 6.0f);
-  const float t = __fmul_rn(q, g);
-  const uint32_t s = cvt_e4m3(t);
-  *scale = s;
-  if (s == 0) {
-    uint32_t packed = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) packed |= ((__float_as_uint(f[i]) >> 31) << 3) << (4 * i);
-    return packed;
-  }
-  const float r = __fdiv_rn(g, e4m3_to_f32(s));
-  float y[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(f[i], r);
-  return cvt_e2m1x8(y);
+// Unsigned division by an invariant divisor d (Granlund and Montgomery,
+// "Division by invariant integers using multiplication", 1994, unsigned
+// case): with l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1,
+// n / d == (mulhi(n, m) + n) >> l for every 32-bit n.
+struct DivU32 {
+  uint32_t m, l;
+};
+
+__device__ __forceinline__ uint32_t div_u32(uint32_t n, DivU32 d) {
+  const uint32_t t = __umulhi(n, d.m);
+  return (uint32_t)(((uint64_t)t + n) >> d.l);
 }
 
+// One thread owns one 16-element block: 32 (bf16) or 64 (f32) contiguous
+// bytes in, 8 bytes of codes and one scale byte out; a warp reads 1 KB
+// (bf16) and writes 256 contiguous bytes of codes.
 template <bool kF32>
-struct Loaded {
-  uint4 v[kF32 ? 2 : 1];
+struct Block16 {
+  uint4 v[kF32 ? 4 : 2];
 };
 
 template <bool kF32>
-__device__ __forceinline__ void load_half(const void* x, int64_t h, Loaded<kF32>& L) {
+__device__ __forceinline__ void load_block(const void* x, uint32_t b, Block16<kF32>& B) {
+  const uint4* p = reinterpret_cast<const uint4*>(x) + (size_t)b * (kF32 ? 4 : 2);
+#pragma unroll
+  for (int i = 0; i < (kF32 ? 4 : 2); ++i) B.v[i] = __ldcs(p + i);
+}
+
+// Largest magnitude of the block.  bf16: clear both sign bits of each packed
+// pair and take the unsigned 16-bit maximum (non-negative bf16 bit patterns
+// order like their values; inputs are finite), then widen exactly to f32.
+template <bool kF32>
+__device__ __forceinline__ float block_amax(const Block16<kF32>& B) {
   if constexpr (kF32) {
-    const uint4* p = reinterpret_cast<const uint4*>(x) + 2 * h;
-    L.v[0] = __ldcs(p);
-    L.v[1] = __ldcs(p + 1);
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      m = fmaxf(m, fabsf(__uint_as_float(B.v[i].x)));
+      m = fmaxf(m, fabsf(__uint_as_float(B.v[i].y)));
+      m = fmaxf(m, fabsf(__uint_as_float(B.v[i].z)));
+      m = fmaxf(m, fabsf(__uint_as_float(B.v[i].w)));
+    }
+    return m;
   } else {
-    L.v[0] = __ldcs(reinterpret_cast<const uint4*>(x) + h);
+    uint32_t w = 0;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      w = __vmaxu2(w, B.v[i].x & 0x7FFF7FFFu);
+      w = __vmaxu2(w, B.v[i].y & 0x7FFF7FFFu);
+      w = __vmaxu2(w, B.v[i].z & 0x7FFF7FFFu);
+      w = __vmaxu2(w, B.v[i].w & 0x7FFF7FFFu);
+    }
+    const uint32_t m16 = max(w >> 16, w & 0xFFFFu);
+    return __uint_as_float(m16 << 16);
   }
 }
 
 template <bool kF32>
-__device__ __forceinline__ void unpack(const Loaded<kF32>& L, float (&f)[8]) {
+__device__ __forceinline__ void block_floats(const Block16<kF32>& B, float (&f)[16]) {
   if constexpr (kF32) {
-    f[0] = __uint_as_float(L.v[0].x); f[1] = __uint_as_float(L.v[0].y);
-    f[2] = __uint_as_float(L.v[0].z); f[3] = __uint_as_float(L.v[0].w);
-    f[4] = __uint_as_float(L.v[1].x); f[5] = __uint_as_float(L.v[1].y);
-    f[6] = __uint_as_float(L.v[1].z); f[7] = __uint_as_float(L.v[1].w);
-  } else {
-    const uint32_t w[4] = {L.v[0].x, L.v[0].y, L.v[0].z, L.v[0].w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      f[2 * i] = __uint_as_float(w[i] << 16);           // bf16 -> f32 is exact
-      f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      f[4 * i + 0] = __uint_as_float(B.v[i].x);
+      f[4 * i + 1] = __uint_as_float(B.v[i].y);
+      f[4 * i + 2] = __uint_as_float(B.v[i].z);
+      f[4 * i + 3] = __uint_as_float(B.v[i].w);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint32_t w[4] = {B.v[i].x, B.v[i].y, B.v[i].z, B.v[i].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        f[8 * i + 2 * k] = __uint_as_float(w[k] << 16);              // bf16 -> f32 is exact
+        f[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+      }
     }
   }
 }
 
-// Grid-stride over "halves" (8-element pieces).  Rows [M, rows_total) only
-// exist in the tensor-core layout (padding to 128 rows): they read nothing
-// and write zero scales.
+// Grid-stride over 16-element blocks.  Blocks of rows [M, rows_total) exist
+// only in the tensor-core layout (rows padded to 128): they read nothing and
+// write zero scales.  rtab[s] = g / e4m3(s) for every scale byte, computed
+// once per CTA with the same correctly rounded division the block formula
+// uses.
 template <bool kF32, bool kTC, bool kAmax>
-__global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ x, int64_t M, int64_t K,
-                                                       int64_t rows_total, float g, uint8_t* __restrict__ codes,
+__global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ x, uint32_t real_blocks,
+                                                       uint32_t total_blocks, uint32_t nblk, DivU32 div_nblk,
+                                                       float g, uint8_t* __restrict__ codes,
                                                        uint8_t* __restrict__ scales, float* amax_out,
                                                        int64_t kc) {
-  constexpr int U = 4;
-  const int lane = threadIdx.x & 31;
-  const int64_t halves_per_row = K >> 3;
-  const int64_t total = rows_total * halves_per_row;   // even: K/8 is even
-  const int64_t real = M * halves_per_row;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  const int64_t nblk = K >> 4;
+  constexpr int U = 2;
+  __shared__ float rtab[256];
+  {
+    const uint32_t s = threadIdx.x;
+    rtab[s] = (s >= 1 && s <= 126) ? __fdiv_rn(g, e4m3_to_f32(s)) : 0.0f;
+  }
+  __syncthreads();
+  const uint32_t stride = gridDim.x * blockDim.x;
   float local_max = 0.0f;
 
-  for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < total; base += U * stride) {
-    Loaded<kF32> L[U];
+  for (uint32_t base = blockIdx.x * blockDim.x + threadIdx.x; base < total_blocks; base += U * stride) {
+    Block16<kF32> B[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int64_t h = base + u * stride + lane;
-      if (h < real) load_half<kF32>(x, h, L[u]);
+      const uint32_t b = base + u * stride;
+      if (b < real_blocks) load_block<kF32>(x, b, B[u]);
       else {
 #pragma unroll
-        for (int i = 0; i < (kF32 ? 2 : 1); ++i) L[u].v[i] = make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < (kF32 ? 4 : 2); ++i) B[u].v[i] = make_uint4(0, 0, 0, 0);
       }
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int64_t h = base + u * stride + lane;
-      float f[8];
-      unpack<kF32>(L[u], f);
-      uint32_t s;
-      float hm;
-      const uint32_t packed = quantize_half_block(f, g, &s, &hm);
-      local_max = fmaxf(local_max, hm);
-      if (h < real) reinterpret_cast<uint32_t*>(codes)[h] = packed;
-      if (h < total && (lane & 1) == 0) {
-        const int64_t row = h / halves_per_row;
-        const int64_t j = (h - row * halves_per_row) >> 1;
-        if constexpr (kTC) {
-          scales[tc_scale_offset(row, j, kc)] = (uint8_t)s;
-          // K % 64 == 32: the last chunk of the row has two padding slots
-          if (j == nblk - 1 && (nblk & 3) == 2) {
-            scales[tc_scale_offset(row, j + 1, kc)] = 0;
-            scales[tc_scale_offset(row, j + 2, kc)] = 0;
-          }
-        } else {
-          scales[row * nblk + j] = (uint8_t)s;
+      const uint32_t b = base + u * stride;
+      if (b >= total_blocks) break;
+      const float amax = block_amax<kF32>(B[u]);
+      if constexpr (kAmax) local_max = fmaxf(local_max, amax);
+      const float q = __fdiv_rn(amax, 6.0f);
+      const float t = __fmul_rn(q, g);
+      const uint32_t s = cvt_e4m3(t);
+      float f[16];
+      block_floats<kF32>(B[u], f);
+      uint32_t lo, hi;
+      if (s == 0) {
+        lo = hi = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          lo |= ((__float_as_uint(f[i]) >> 31) << 3) << (4 * i);
+          hi |= ((__float_as_uint(f[8 + i]) >> 31) << 3) << (4 * i);
         }
+      } else {
+        const float r = rtab[s];
+        float y0[8], y1[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          y0[i] = __fmul_rn(f[i], r);
+          y1[i] = __fmul_rn(f[8 + i], r);
+        }
+        lo = cvt_e2m1x8(y0);
+        hi = cvt_e2m1x8(y1);
+      }
+      if (b < real_blocks) reinterpret_cast<uint2*>(codes)[b] = make_uint2(lo, hi);
+      if constexpr (kTC) {
+        const uint32_t row = div_u32(b, div_nblk);
+        const uint32_t j = b - row * nblk;
+        scales[tc_scale_offset(row, j, kc)] = (uint8_t)s;
+        // K % 64 == 32: the last chunk of the row has two padding slots
+        if (j == nblk - 1 && (nblk & 3) == 2) {
+          scales[tc_scale_offset(row, j + 1, kc)] = 0;
+          scales[tc_scale_offset(row, j + 2, kc)] = 0;
+        }
+      } else {
+        scales[b] = (uint8_t)s;
       }
     }
   }
 
   if constexpr (kAmax) {
+    const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) local_max = fmaxf(local_max, __shfl_xor_sync(0xFFFFFFFFu, local_max, o));
     __shared__ float wmax[8];
     if (lane == 0) wmax[threadIdx.x >> 5] = local_max;
     __syncthreads();
     if (threadIdx.x == 0) {
-      float b = 0.0f;
-      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) b = fmaxf(b, wmax[w]);
+      float bmax = 0.0f;
+      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) bmax = fmaxf(bmax, wmax[w]);
       // non-negative floats order like their bit patterns
-      atomicMax(reinterpret_cast<unsigned*>(amax_out), __float_as_uint(b));
+      atomicMax(reinterpret_cast<unsigned*>(amax_out), __float_as_uint(bmax));
     }
   }
 }
@@ -271,18 +316,29 @@ int grid_for(int64_t work_items, int threads, const DeviceInfo* d, int per_sm = 
   return (int)blocks;
 }
 
+DivU32 make_div(uint32_t d) {
+  uint32_t l = 0;
+  while ((1ull << l) < d) ++l;
+  DivU32 r;
+  r.l = l;
+  r.m = (uint32_t)((((1ull << l) - d) << 32) / d + 1);
+  return r;
+}
+
 template <bool kF32, bool kTC, bool kAmax>
 cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, float g, uint8_t* codes, uint8_t* scales,
                             float* amax_out, cudaStream_t st, const DeviceInfo* d) {
   const int64_t rows_total = kTC ? ceil_div(M, 128) * 128 : M;
   const int64_t kc = ceil_div(K, 64);
-  const int64_t halves = rows_total * (K / 8);
-  // each warp-iteration covers U*stride halves; size the grid so every SM
-  // holds 2048 threads when there is enough work
+  const uint32_t nblk = (uint32_t)(K / 16);
+  const uint32_t real = (uint32_t)(M * (K / 16));
+  const uint32_t total = (uint32_t)(rows_total * (K / 16));
+  // 256 threads, 2 blocks of 16 elements per thread per iteration, up to 8
+  // CTAs (2048 threads) per SM
   const int threads = 256;
-  int blocks = grid_for(ceil_div(halves, 4), threads, d, 8);
-  quantize_kernel<kF32, kTC, kAmax><<<blocks, threads, 0, st>>>(x, M, K, rows_total, g, codes, scales,
-                                                                amax_out, kc);
+  const int blocks = grid_for(ceil_div(total, 2), threads, d, 8);
+  quantize_kernel<kF32, kTC, kAmax><<<blocks, threads, 0, st>>>(x, real, total, nblk, make_div(nblk), g, codes,
+                                                                scales, amax_out, kc);
   return cudaGetLastError();
 }
 
@@ -324,6 +380,7 @@ nvfp4_status nvfp4_quantize(const void* x, nvfp4_in_dtype dtype, int64_t M, int6
                             nvfp4_stream_t stream) {
   if (!x || !codes || !block_scales || M < 1 || K < 32 || K % 32 != 0) return NVFP4_ERR_INVALID_ARG;
   if (dtype != NVFP4_IN_BF16 && dtype != NVFP4_IN_F32) return NVFP4_ERR_INVALID_ARG;
+  if (ceil_div(M, 128) * 128 * (K / 16) >= (1ll << 31)) return NVFP4_ERR_UNSUPPORTED;
   if (layout != NVFP4_SF_ROWMAJOR && layout != NVFP4_SF_TCGEN05) return NVFP4_ERR_INVALID_ARG;
   if (!finite_positive(global_scale)) return NVFP4_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(codes) || !aligned16(block_scales)) return NVFP4_ERR_ALIGNMENT;

@@ -160,3 +160,18 @@ def test_output_guard_bands_untouched():
     nv.nvfp4_gemm(a_d, as_d, float(ga), w_d, ws_d, float(gw), M, N, K, out)
     torch.cuda.synchronize()
     assert torch.all(buf[:pad] == -7.0) and torch.all(buf[pad + M * N:] == -7.0)
+
+
+@pytest.mark.parametrize("M,N,K", [(200, 128, 512), (300, 48, 256), (260, 320, 512), (131, 72, 320)])
+def test_gemm_partial_last_tile_bf16(M, N, K):
+    # normal tiles whose last 64-column output sub-tiles fall past N: the
+    # bf16 result must still be bf16(f32 result) everywhere
+    (ac, asc, ga), (wc, wsc, gw) = _operands(M, N, K, seed=M * N + K)
+    ref = oracle.gemm(ac, asc, ga, wc, wsc, gw)
+    a_d, as_d = to_dev_operand(ac, asc, K)
+    w_d, ws_d = to_dev_operand(wc, wsc, K)
+    for _ in range(3):
+        out32 = gpu_gemm(a_d, as_d, ga, w_d, ws_d, gw, M, N, K, torch.float32)
+        out16 = gpu_gemm(a_d, as_d, ga, w_d, ws_d, gw, M, N, K, torch.bfloat16)
+        assert torch.equal(out16, out32.to(torch.bfloat16))
+    assert_gemm_close(out32.cpu().numpy(), ref, f"{M}x{N}x{K}")
