@@ -94,13 +94,23 @@ struct Cfg {
   static constexpr int kOffSeg = kOffBar + kNumBars * 8;             // segment table: ends, alphas
   static constexpr int kOffMisc = kOffSeg + 2 * 4 * NVFP4_MAX_SEGMENTS;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;            // + alignment slack
-  // TMEM columns: accumulator, then per-stage scale regions
+  // TMEM columns.  Normal 128x256 tiles: two accumulator buffers, [0,256)
+  // and [192,448), overlapping in 64 columns, so tile t+1 can start as soon
+  // as the epilogue has drained the 64 shared columns of tile t; the scale
+  // factors of the stage being computed sit in [448,496) (tcgen05 operations
+  // of one thread execute in issue order, so one scale region serves every
+  // stage).  Swapped (decode) tiles: one accumulator and one scale region per
+  // pipeline stage.
   static constexpr int kAccCols = BN < 32 ? 32 : BN;
+  static constexpr bool kOverlapAcc = !SWAP && BN == 256;
+  static constexpr int kAcc1Col = kOverlapAcc ? 192 : 0;
   static constexpr int kSfaCols = 16;                                // 4 MMAs x 4 columns
   static constexpr int kSfbCols = kSfbBlocks * 16;
   static constexpr int kSfStageCols = kSfaCols + kSfbCols;
+  static constexpr int kSfBase = kOverlapAcc ? 448 : kAccCols;
+  static constexpr int kSfRegions = kOverlapAcc ? 1 : kStages;
   static_assert(kStages >= 2, "pipeline depth");
-  static_assert(kAccCols + kStages * kSfStageCols <= kTmemCols, "TMEM budget");
+  static_assert(kSfBase + kSfRegions * kSfStageCols <= kTmemCols, "TMEM budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(BN % 16 == 0 && BN <= 256, "MMA N");
 };
@@ -238,19 +248,19 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
       const uint64_t b_desc0 = smem_desc(sbase + C::kOffB, 16, 1024, 2);
       const uint64_t sfa_desc0 = smem_desc(sbase + C::kOffSfa, 16, 128, 0);
       const uint64_t sfb_desc0 = smem_desc(sbase + C::kOffSfb, 16, 128, 0);
-      const uint32_t acc = tmem_base;
-      const uint32_t sf_t0 = tmem_base + C::kAccCols;
+      const uint32_t sf_t0 = tmem_base + C::kSfBase;
       const int kt = p.kt, kc = p.kc;
       int stage = 0;
-      uint32_t phase = 0, acc_phase = 0;
+      uint32_t phase = 0, acc_phase = 0, acc_buf = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
         if (!mbar_wait(bar_acc_empty, acc_phase ^ 1, abort_flag, p.err, p.timeout_ns)) break;
         tc_fence_after();
+        const uint32_t acc = tmem_base + (acc_buf ? C::kAcc1Col : 0);
         for (int k = 0; k < kt; ++k) {
           if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, p.err, p.timeout_ns)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sfa_t = sf_t0 + stage * C::kSfStageCols;
+          const uint32_t sfa_t = sf_t0 + (C::kSfRegions == 1 ? 0 : stage) * C::kSfStageCols;
           const uint32_t sfb_t = sfa_t + C::kSfaCols;
           const uint64_t ad = a_desc0 + (uint64_t)((stage * C::kABytes) >> 4);
           const uint64_t bd = b_desc0 + (uint64_t)((stage * C::kBBytes) >> 4);
@@ -289,6 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
         if (!ok) break;
         tc_commit(bar_acc_full);
         acc_phase ^= 1;
+        acc_buf ^= 1;
       }
       // every MMA and scale copy issued by this thread has completed once
       // this commit arrives
@@ -306,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
     const int n_seg = p.n_seg;
     const float alpha0 = seg_alpha_s[0];
     const bool tma_store = !SWAP && p.tma_store;
-    uint32_t acc_phase = 0;
+    uint32_t acc_phase = 0, acc_buf = 0;
     uint32_t out_buf = 0;                    // next staging buffer (TMA store path)
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
       int tp, tq;
@@ -317,38 +328,55 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
       tc_fence_after();
       if constexpr (!SWAP) {
         const int64_t m = p0 + row;
+        // 64-column slots are drained starting with the columns this buffer
+        // shares with the other one; TMEM is handed back right after them.
+        const uint32_t tacc = taddr + (acc_buf ? C::kAcc1Col : 0);
+        auto slot_col = [&](int slot) -> int {
+          return C::kOverlapAcc && acc_buf == 0 ? ((slot + 3) & 3) * 64 : slot * 64;
+        };
         if constexpr (!OUT_F32) {
-          // drain the whole accumulator row into registers (bf16 pairs), then
-          // hand TMEM back to the MMA warp before any store
+          // drain the whole accumulator row into registers (bf16 pairs)
           uint32_t packed[BN / 2];
 #pragma unroll
-          for (int c = 0; c < BN / 32; c += 2) {
+          for (int slot = 0; slot < BN / 64; ++slot) {
+            const int col = slot_col(slot);
             uint32_t r0[32], r1[32];
-            tmem_ld_32x32b_x32(taddr + c * 32, r0);
-            tmem_ld_32x32b_x32(taddr + (c + 1) * 32, r1);
+            tmem_ld_32x32b_x32(tacc + col, r0);
+            tmem_ld_32x32b_x32(tacc + col + 32, r1);
             tmem_ld_wait();
-            float a[2] = {alpha0, alpha0};
-            const bool seg_uniform =
-                n_seg == 1 || seg_index_smem(seg_end_s, n_seg, q0 + c * 32) ==
-                                  seg_index_smem(seg_end_s, n_seg, q0 + c * 32 + 63);
-            if (seg_uniform) a[0] = a[1] = seg_alpha_smem(seg_end_s, seg_alpha_s, n_seg, q0 + c * 32);
+            if (slot == 0 && C::kOverlapAcc) {
+              tc_fence_before();
+              mbar_arrive(bar_acc_empty);
+            }
+            const int64_t n0 = q0 + col;
+            if (n_seg == 1) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float alo = a[0], ahi = a[0], blo = a[1], bhi = a[1];
-              if (!seg_uniform) {
-                alo = seg_alpha_smem(seg_end_s, seg_alpha_s, n_seg, q0 + c * 32 + 2 * i);
-                ahi = seg_alpha_smem(seg_end_s, seg_alpha_s, n_seg, q0 + c * 32 + 2 * i + 1);
-                blo = seg_alpha_smem(seg_end_s, seg_alpha_s, n_seg, q0 + c * 32 + 32 + 2 * i);
-                bhi = seg_alpha_smem(seg_end_s, seg_alpha_s, n_seg, q0 + c * 32 + 33 + 2 * i);
+              for (int i = 0; i < 16; ++i) {
+                packed[slot * 32 + i] = pack_bf16x2(__fmul_rn(__uint_as_float(r0[2 * i]), alpha0),
+                                                    __fmul_rn(__uint_as_float(r0[2 * i + 1]), alpha0));
+                packed[slot * 32 + 16 + i] = pack_bf16x2(__fmul_rn(__uint_as_float(r1[2 * i]), alpha0),
+                                                         __fmul_rn(__uint_as_float(r1[2 * i + 1]), alpha0));
               }
-              packed[c * 16 + i] = pack_bf16x2(__fmul_rn(__uint_as_float(r0[2 * i]), alo),
-                                               __fmul_rn(__uint_as_float(r0[2 * i + 1]), ahi));
-              packed[(c + 1) * 16 + i] = pack_bf16x2(__fmul_rn(__uint_as_float(r1[2 * i]), blo),
-                                                     __fmul_rn(__uint_as_float(r1[2 * i + 1]), bhi));
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                packed[slot * 32 + i] =
+                    pack_bf16x2(__fmul_rn(__uint_as_float(r0[2 * i]),
+                                          seg_alpha_smem(seg_end_s, seg_alpha_s, n_seg, n0 + 2 * i)),
+                                __fmul_rn(__uint_as_float(r0[2 * i + 1]),
+                                          seg_alpha_smem(seg_end_s, seg_alpha_s, n_seg, n0 + 2 * i + 1)));
+                packed[slot * 32 + 16 + i] =
+                    pack_bf16x2(__fmul_rn(__uint_as_float(r1[2 * i]),
+                                          seg_alpha_smem(seg_end_s, seg_alpha_s, n_seg, n0 + 32 + 2 * i)),
+                                __fmul_rn(__uint_as_float(r1[2 * i + 1]),
+                                          seg_alpha_smem(seg_end_s, seg_alpha_s, n_seg, n0 + 33 + 2 * i)));
+              }
             }
           }
-          tc_fence_before();
-          mbar_arrive(bar_acc_empty);
+          if (!C::kOverlapAcc) {
+            tc_fence_before();
+            mbar_arrive(bar_acc_empty);
+          }
           if (tma_store) {
             // 64-column sub-tiles through two 16 KB swizzled staging buffers
 #pragma unroll
@@ -356,7 +384,8 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
               // sub-tiles wholly past N are skipped outright (uniform across
               // the epilogue), so every buffer written is one whose last
               // store has been committed and waited for
-              if (q0 + sub * 64 >= N) continue;
+              const int col = slot_col(sub);
+              if (q0 + col >= N) continue;
               const uint32_t buf = sbase + C::kOffOut + out_buf * kStageOutBytes;
               if (et == 0) bulk_wait_group_read<1>();          // the store that used buf has read it
               named_bar_sync(kEpiBar, 128);
@@ -370,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
               fence_proxy_async_smem();
               named_bar_sync(kEpiBar, 128);
               if (et == 0) {
-                tma_store_2d(&p.tmap_out, buf, (int32_t)(q0 + sub * 64), (int32_t)p0);
+                tma_store_2d(&p.tmap_out, buf, (int32_t)(q0 + col), (int32_t)p0);
                 bulk_commit_group();
               }
               out_buf ^= 1;
@@ -379,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
             __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) + m * N;
 #pragma unroll
             for (int c = 0; c < BN / 8; ++c) {
-              const int64_t n = q0 + c * 8;
+              const int64_t n = q0 + slot_col(c / 8) + (c % 8) * 8;
 #pragma unroll
               for (int e = 0; e < 8; ++e)
                 if (n + e < N)
@@ -387,13 +416,19 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
             }
           }
         } else {
-          // FP32 output: 32-column chunks; TMEM is released after the last one
+          // FP32 output: 32-column chunks in slot order; TMEM is released once
+          // the shared columns (the first slot) are out
 #pragma unroll 1
-          for (int c = 0; c < BN / 32; ++c) {
+          for (int cc = 0; cc < BN / 32; ++cc) {
+            const int c = slot_col(cc / 2) / 32 + (cc & 1);
             uint32_t r[32];
             __syncwarp();
-            tmem_ld_32x32b_x32(taddr + c * 32, r);
+            tmem_ld_32x32b_x32(tacc + c * 32, r);
             tmem_ld_wait();
+            if (cc == 1 && C::kOverlapAcc) {
+              tc_fence_before();
+              mbar_arrive(bar_acc_empty);
+            }
 #pragma unroll
             for (int i = 0; i < 32; ++i)
               r[i] = __float_as_uint(
@@ -423,8 +458,10 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
               }
             }
           }
-          tc_fence_before();
-          mbar_arrive(bar_acc_empty);
+          if (!C::kOverlapAcc) {
+            tc_fence_before();
+            mbar_arrive(bar_acc_empty);
+          }
         }
       } else {
         // swap: lane = weight row = output column n; accumulator column = activation row
@@ -462,6 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
         mbar_arrive(bar_acc_empty);
       }
       acc_phase ^= 1;
+      acc_buf ^= 1;
     }
     if (tma_store && et == 0) bulk_wait_group<0>();   // stores done before the CTA's smem goes away
   }
