@@ -21,7 +21,13 @@
  * Conventions shared by every entry point
  *   - Device pointers are raw CUDA device addresses owned by the caller; the
  *     library never allocates, frees or retains them.  Host pointers (named
- *     so below) are read during the call only.
+ *     so below) are read during the call only.  The one buffer the library
+ *     owns is the GEMM's K-split workspace (see nvfp4_gemm).
+ *   - Consecutive kernels of this library on one stream overlap their
+ *     prologue with the previous kernel's tail (programmatic dependent
+ *     launch); each still reads its inputs only after the kernel before it
+ *     on the stream has completed, so stream order is the only ordering
+ *     callers need.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and the call returns once enqueued; nothing synchronizes.
  *   - Arguments are validated before anything is launched.  A failing check
@@ -132,7 +138,18 @@ NVFP4_API nvfp4_status nvfp4_swizzle_scales(const uint8_t* rowmajor, int64_t row
  *   out     device [M, N] row-major, bf16 or f32 per out_dtype
  * All device pointers 16-byte aligned; M, N >= 1; K >= 32, K % 32 == 0;
  * global scales finite and > 0.
- * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (device is not sm_100), CUDA. */
+ * For M <= 128 (decode) the K loop of each weight tile is split across CTAs
+ * so that every SM streams weight; the partial FP32 tiles are summed in a
+ * fixed order (the result does not depend on timing and equals the unsplit
+ * sum up to FP32 rounding order).  The partials go to a workspace the
+ * library allocates on first use for each (device, stream) pair
+ * (2 * SMs * 64 KB plus 256 KB of counters) and keeps until the process
+ * exits.  That first call on a stream must not be made while the stream is
+ * being captured into a CUDA graph: it returns UNSUPPORTED then.  Calls on
+ * one stream share its workspace safely (stream order); calls on different
+ * streams use different workspaces.
+ * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (device is not sm_100, or a
+ * first decode-shaped call during capture), CUDA. */
 NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float a_global_scale,
                         const uint8_t* w_codes, const uint8_t* w_scales, float w_global_scale,
                         int64_t M, int64_t N, int64_t K, void* out, nvfp4_out_dtype out_dtype,

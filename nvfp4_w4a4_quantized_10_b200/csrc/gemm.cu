@@ -35,7 +35,9 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "common.h"
 #include "ptx.cuh"
@@ -58,6 +60,8 @@ struct alignas(64) GemmParams {
   const uint8_t* sf_p;
   const uint8_t* sf_q;
   void* out;
+  float* ws;             // swapped tiles: FP32 partial tiles, 2 slots per CTA
+  int* tickets;          // swapped tiles: per-tile arrival counters (zero between launches)
   unsigned* err;
   uint64_t timeout_ns;
   int64_t M, N;          // output [M, N]
@@ -130,6 +134,58 @@ __device__ __forceinline__ void tile_coords(const GemmParams& p, int tile, int& 
   tq = local / gsize;
 }
 
+// Work of one CTA, as a sequence of (tile, k-step range) items.
+//   normal tiles: whole tiles t = blockIdx.x, blockIdx.x + gridDim.x, ...
+//   swapped tiles (stream-K): the tiles_p * kt (tile, k-step) units are cut
+//   into gridDim.x contiguous, balanced ranges; CTA c owns units
+//   [floor(c U / G), floor((c+1) U / G)).  An item is the part of that range
+//   inside one tile.
+struct WorkIter {
+  int64_t u, u_end;   // swapped: unit range; normal: next tile index, tile count
+  int kt;
+  bool swap;
+};
+
+__device__ __forceinline__ int64_t unit_begin(int64_t c, int64_t U, int64_t G) { return c * U / G; }
+
+// CTA whose range holds unit u: the largest c with floor(c U / G) <= u.
+__device__ __forceinline__ int64_t cta_of_unit(int64_t u, int64_t U, int64_t G) {
+  return ((u + 1) * G + U - 1) / U - 1;
+}
+
+__device__ __forceinline__ WorkIter work_begin(const GemmParams& p, bool swap) {
+  WorkIter w;
+  w.kt = p.kt;
+  w.swap = swap;
+  if (swap) {
+    const int64_t U = (int64_t)p.tiles_p * p.kt, G = gridDim.x;
+    w.u = unit_begin(blockIdx.x, U, G);
+    w.u_end = unit_begin(blockIdx.x + 1, U, G);
+  } else {
+    w.u = blockIdx.x;
+    w.u_end = (int64_t)p.tiles_p * p.tiles_q;
+  }
+  return w;
+}
+
+__device__ __forceinline__ bool work_next(const GemmParams& p, WorkIter& w, int& tp, int& tq, int& kb, int& ke) {
+  if (w.u >= w.u_end) return false;
+  if (w.swap) {
+    tp = (int)(w.u / w.kt);
+    tq = 0;
+    kb = (int)(w.u - (int64_t)tp * w.kt);
+    const int64_t rest = w.u_end - w.u;
+    ke = (int)(kb + rest < w.kt ? kb + rest : w.kt);
+    w.u += ke - kb;
+  } else {
+    tile_coords(p, (int)w.u, tp, tq);
+    kb = 0;
+    ke = w.kt;
+    w.u += gridDim.x;
+  }
+  return true;
+}
+
 // Segment of output column n, from the table the CTA copied to shared memory.
 __device__ __forceinline__ int seg_index_smem(const int* ends, int n_seg, int64_t n) {
   int i = 0;
@@ -160,10 +216,13 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
   float* seg_alpha_s = reinterpret_cast<float*>(smem + C::kOffSeg + 4 * NVFP4_MAX_SEGMENTS);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int total_tiles = p.tiles_p * p.tiles_q;
+  // the next kernel in the stream may launch now; it waits for this grid's
+  // completion before touching anything this grid reads or writes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -194,40 +253,76 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // The weight operand (P when swapped, Q otherwise) does not depend on
+    // the preceding kernel, so the weight side of the first kStages steps is
+    // requested before waiting on it (programmatic dependent launch); every
+    // activation load comes after griddepcontrol.wait.
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
+      const int kc = p.kc, rb_q = p.rb_q;
       uint32_t issued_mask = 0, last_parity = 0;   // for the drain on abort
       bool ok = true;
-      const int kt = p.kt, kc = p.kc, rb_q = p.rb_q;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-        int tp, tq;
-        tile_coords(p, tile, tp, tq);
-        const int p0 = tp * kBM, q0 = tq * BN;
-        const uint8_t* sfp = p.sf_p + (size_t)(p0 >> 7) * kc * kSfChunk;
-        const uint8_t* sfq = p.sf_q + (size_t)(q0 >> 7) * kc * kSfChunk;
-        int nsfb = 0;
+      auto for_steps = [&](WorkIter w, int first, int count, auto&& fn) {
+        int tp, tq, kb, ke, j = 0;
+        while (j < first + count && work_next(p, w, tp, tq, kb, ke))
+          for (int k = kb; k < ke && j < first + count; ++k, ++j)
+            if (j >= first) fn(j, tp * kBM, tq * BN, k);
+      };
+      auto nsfb_of = [&](int q0) {
+        int n = 0;
 #pragma unroll
         for (int rb = 0; rb < C::kSfbBlocks; ++rb)
-          if ((q0 >> 7) + rb < rb_q) ++nsfb;
-        for (int k = 0; k < kt; ++k) {
-          if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, p.err, p.timeout_ns)) { ok = false; break; }
-          const int nch = min(4, kc - 4 * k);
-          const uint32_t sf_bytes = (uint32_t)nch * kSfChunk;
-          const uint32_t fb = bar_full + 8 * stage;
-          mbar_arrive_expect_tx(fb, C::kABytes + C::kBBytes + sf_bytes * (1 + nsfb));
-          tma_load_2d(sbase + C::kOffA + stage * C::kABytes, &p.tmap_p, k * kBKBytes, p0, fb);
-          tma_load_2d(sbase + C::kOffB + stage * C::kBBytes, &p.tmap_q, k * kBKBytes, q0, fb);
-          bulk_load(sbase + C::kOffSfa + stage * C::kSfaBytes, sfp + (size_t)(4 * k) * kSfChunk, sf_bytes, fb);
+          if ((q0 >> 7) + rb < rb_q) ++n;
+        return n;
+      };
+      auto load_p = [&](int stage, int p0, int k) {
+        const uint32_t fb = bar_full + 8 * stage;
+        const uint32_t sf_bytes = (uint32_t)min(4, kc - 4 * k) * kSfChunk;
+        tma_load_2d(sbase + C::kOffA + stage * C::kABytes, &p.tmap_p, k * kBKBytes, p0, fb);
+        bulk_load(sbase + C::kOffSfa + stage * C::kSfaBytes,
+                  p.sf_p + ((size_t)(p0 >> 7) * kc + 4 * k) * kSfChunk, sf_bytes, fb);
+      };
+      auto load_q = [&](int stage, int q0, int k) {
+        const uint32_t fb = bar_full + 8 * stage;
+        const uint32_t sf_bytes = (uint32_t)min(4, kc - 4 * k) * kSfChunk;
+        const int nsfb = nsfb_of(q0);
+        tma_load_2d(sbase + C::kOffB + stage * C::kBBytes, &p.tmap_q, k * kBKBytes, q0, fb);
 #pragma unroll
-          for (int rb = 0; rb < C::kSfbBlocks; ++rb)
-            if (rb < nsfb)
-              bulk_load(sbase + C::kOffSfb + stage * C::kSfbBytes + rb * 4 * kSfChunk,
-                        sfq + ((size_t)rb * kc + 4 * k) * kSfChunk, sf_bytes, fb);
-          issued_mask |= 1u << stage;
+        for (int rb = 0; rb < C::kSfbBlocks; ++rb)
+          if (rb < nsfb)
+            bulk_load(sbase + C::kOffSfb + stage * C::kSfbBytes + rb * 4 * kSfChunk,
+                      p.sf_q + ((size_t)((q0 >> 7) + rb) * kc + 4 * k) * kSfChunk, sf_bytes, fb);
+      };
+      auto expect = [&](int stage, int q0, int k) {
+        const uint32_t sf_bytes = (uint32_t)min(4, kc - 4 * k) * kSfChunk;
+        mbar_arrive_expect_tx(bar_full + 8 * stage, C::kABytes + C::kBBytes + sf_bytes * (1 + nsfb_of(q0)));
+      };
+      const WorkIter w0 = work_begin(p, SWAP);
+      // prologue: the first kStages stages are free
+      int npro = 0;
+      for_steps(w0, 0, C::kStages, [&](int j, int p0, int q0, int k) {
+        expect(j, q0, k);
+        if (SWAP) load_p(j, p0, k);
+        else load_q(j, q0, k);
+        issued_mask |= 1u << j;
+        npro = j + 1;
+      });
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      for_steps(w0, 0, npro, [&](int j, int p0, int q0, int k) {
+        if (SWAP) load_q(j, q0, k);
+        else load_p(j, p0, k);
+      });
+      int stage = npro % C::kStages;
+      uint32_t phase = npro == C::kStages ? 1u : 0u;
+      if (npro == C::kStages) {
+        for_steps(w0, npro, 1 << 30, [&](int j, int p0, int q0, int k) {
+          if (!ok) return;
+          if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, p.err, p.timeout_ns)) { ok = false; return; }
+          expect(stage, q0, k);
+          load_p(stage, p0, k);
+          load_q(stage, q0, k);
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
-        }
+        });
       }
       if (*abort_flag) {
         // let every issued copy land before the CTA exits
@@ -240,73 +335,82 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_nvf4(kBM, BN);
-      // Descriptors of stage 0, k-block 0; later stages and k-blocks only move
-      // the 14-bit start-address field (address >> 4), which never carries.
-      const uint64_t a_desc0 = smem_desc(sbase + C::kOffA, 16, 1024, 2);
-      const uint64_t b_desc0 = smem_desc(sbase + C::kOffB, 16, 1024, 2);
-      const uint64_t sfa_desc0 = smem_desc(sbase + C::kOffSfa, 16, 128, 0);
-      const uint64_t sfb_desc0 = smem_desc(sbase + C::kOffSfb, 16, 128, 0);
-      const uint32_t sf_t0 = tmem_base + C::kSfBase;
-      const int kt = p.kt, kc = p.kc;
-      int stage = 0;
-      uint32_t phase = 0, acc_phase = 0, acc_buf = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-        if (!mbar_wait(bar_acc_empty, acc_phase ^ 1, abort_flag, p.err, p.timeout_ns)) break;
+    // The whole warp follows the pipeline; lane 0 issues every tcgen05 operation.
+    constexpr uint32_t idesc = idesc_nvf4(kBM, BN);
+    // Descriptors of stage 0, k-block 0; later stages and k-blocks only move
+    // the 14-bit start-address field (address >> 4), which never carries.
+    const uint64_t a_desc0 = smem_desc(sbase + C::kOffA, 16, 1024, 2);
+    const uint64_t b_desc0 = smem_desc(sbase + C::kOffB, 16, 1024, 2);
+    const uint64_t sfa_desc0 = smem_desc(sbase + C::kOffSfa, 16, 128, 0);
+    const uint64_t sfb_desc0 = smem_desc(sbase + C::kOffSfb, 16, 128, 0);
+    const uint32_t sf_t0 = tmem_base + C::kSfBase;
+    const int kc = p.kc;
+    int stage = 0;
+    uint32_t phase = 0, acc_phase = 0, acc_buf = 0;
+    bool ok = true;
+    WorkIter w = work_begin(p, SWAP);
+    int tp, tq, kb0, ke0;
+    while (ok && work_next(p, w, tp, tq, kb0, ke0)) {
+      if (!mbar_wait(bar_acc_empty, acc_phase ^ 1, abort_flag, p.err, p.timeout_ns)) break;
+      tc_fence_after();
+      const uint32_t acc = tmem_base + (acc_buf ? C::kAcc1Col : 0);
+      for (int k = kb0; k < ke0; ++k) {
+        if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, p.err, p.timeout_ns)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t acc = tmem_base + (acc_buf ? C::kAcc1Col : 0);
-        for (int k = 0; k < kt; ++k) {
-          if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, p.err, p.timeout_ns)) { ok = false; break; }
-          tc_fence_after();
+        const uint32_t sb = sbase + C::kOffSfb + stage * C::kSfbBytes;
+        if (lane == 0) {
           const uint32_t sfa_t = sf_t0 + (C::kSfRegions == 1 ? 0 : stage) * C::kSfStageCols;
           const uint32_t sfb_t = sfa_t + C::kSfaCols;
           const uint64_t ad = a_desc0 + (uint64_t)((stage * C::kABytes) >> 4);
           const uint64_t bd = b_desc0 + (uint64_t)((stage * C::kBBytes) >> 4);
           const uint64_t sad = sfa_desc0 + (uint64_t)((stage * C::kSfaBytes) >> 4);
           const uint64_t sbd = sfb_desc0 + (uint64_t)((stage * C::kSfbBytes) >> 4);
-          const uint32_t acc_in = k != 0 ? 1u : 0u;
+          const uint32_t acc_in = k != kb0 ? 1u : 0u;
+          // TMEM column of Q's scales for K-block kb (multiples of 4 columns)
+          auto sfq_col = [&](int kb, int rb) -> uint32_t { return sfb_t + kb * 4 * C::kSfbBlocks + rb * 4; };
           if (4 * k + 4 <= kc) {
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb) {
               tc_cp_32x128b_warpx4(sfa_t + kb * 4, sad + (uint64_t)(kb * (kSfChunk >> 4)));
 #pragma unroll
               for (int rb = 0; rb < C::kSfbBlocks; ++rb)
-                tc_cp_32x128b_warpx4(sfb_t + kb * 4 * C::kSfbBlocks + rb * 4,
-                                     sbd + (uint64_t)((rb * 4 + kb) * (kSfChunk >> 4)));
+                tc_cp_32x128b_warpx4(sfq_col(kb, rb), sbd + (uint64_t)((rb * 4 + kb) * (kSfChunk >> 4)));
             }
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb)
               tc_mma_nvf4(acc, ad + (uint64_t)(kb * 2), bd + (uint64_t)(kb * 2), idesc, sfa_t + kb * 4,
-                          sfb_t + kb * 4 * C::kSfbBlocks, (acc_in | kb) != 0 ? 1u : 0u);
+                          sfq_col(kb, 0), (acc_in | kb) != 0 ? 1u : 0u);
           } else {
             const int nkb = kc - 4 * k;
             for (int kb = 0; kb < nkb; ++kb) {
               tc_cp_32x128b_warpx4(sfa_t + kb * 4, sad + (uint64_t)(kb * (kSfChunk >> 4)));
 #pragma unroll
               for (int rb = 0; rb < C::kSfbBlocks; ++rb)
-                tc_cp_32x128b_warpx4(sfb_t + kb * 4 * C::kSfbBlocks + rb * 4,
-                                     sbd + (uint64_t)((rb * 4 + kb) * (kSfChunk >> 4)));
+                tc_cp_32x128b_warpx4(sfq_col(kb, rb), sbd + (uint64_t)((rb * 4 + kb) * (kSfChunk >> 4)));
             }
             for (int kb = 0; kb < nkb; ++kb)
               tc_mma_nvf4(acc, ad + (uint64_t)(kb * 2), bd + (uint64_t)(kb * 2), idesc, sfa_t + kb * 4,
-                          sfb_t + kb * 4 * C::kSfbBlocks, (acc_in | kb) != 0 ? 1u : 0u);
+                          sfq_col(kb, 0), (acc_in | kb) != 0 ? 1u : 0u);
           }
           tc_commit(bar_empty + 8 * stage);
-          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
-        if (!ok) break;
-        tc_commit(bar_acc_full);
-        acc_phase ^= 1;
-        acc_buf ^= 1;
+        __syncwarp();
+        if (++stage == C::kStages) { stage = 0; phase ^= 1; }
       }
+      if (!ok) break;
+      if (lane == 0) tc_commit(bar_acc_full);
+      __syncwarp();
+      acc_phase ^= 1;
+      acc_buf ^= 1;
+    }
+    if (lane == 0) {
       // every MMA and scale copy issued by this thread has completed once
       // this commit arrives
       tc_commit(bar_drain);
       volatile int never = 0;
       (void)mbar_wait(bar_drain, 0, &never, p.err, p.timeout_ns);
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
     const int sp = warp & 3;                 // TMEM subpartition of this warp
@@ -319,9 +423,11 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
     const bool tma_store = !SWAP && p.tma_store;
     uint32_t acc_phase = 0, acc_buf = 0;
     uint32_t out_buf = 0;                    // next staging buffer (TMA store path)
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-      int tp, tq;
-      tile_coords(p, tile, tp, tq);
+    WorkIter w = work_begin(p, SWAP);
+    const int64_t U = (int64_t)p.tiles_p * p.kt, G = gridDim.x;
+    int tp, tq, kb0, ke0;
+    bool first_item = true;
+    while (work_next(p, w, tp, tq, kb0, ke0)) {
       const int64_t p0 = (int64_t)tp * kBM, q0 = (int64_t)tq * BN;
       if (!mbar_wait(bar_acc_full, acc_phase, abort_flag, p.err, p.timeout_ns)) break;
       __syncwarp();
@@ -464,42 +570,121 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
           }
         }
       } else {
-        // swap: lane = weight row = output column n; accumulator column = activation row
+        // swap: lane = weight row = output column n; accumulator column =
+        // activation row.  The whole accumulator row goes to registers, then
+        // TMEM is handed back.
         const int64_t n = p0 + row;
         const float alpha = seg_alpha_smem(seg_end_s, seg_alpha_s, n_seg, n);
+        constexpr int kCols = BN < 32 ? BN : 32;
+        uint32_t r[(BN + 31) / 32][kCols];
 #pragma unroll
         for (int c = 0; c < (BN + 31) / 32; ++c) {
-          uint32_t r[32];
-          __syncwarp();
           if constexpr (BN >= 32) {
-            tmem_ld_32x32b_x32(taddr + c * 32, r);
+            tmem_ld_32x32b_x32(taddr + c * 32, r[c]);
           } else {
             uint32_t r8[8];
 #pragma unroll
             for (int j = 0; j < BN / 8; ++j) {
               tmem_ld_32x32b_x8(taddr + j * 8, r8);
 #pragma unroll
-              for (int i = 0; i < 8; ++i) r[j * 8 + i] = r8[i];
-            }
-          }
-          tmem_ld_wait();
-          if (n < N) {
-#pragma unroll
-            for (int i = 0; i < (BN < 32 ? BN : 32); ++i) {
-              const int64_t mm = q0 + c * 32 + i;
-              if (mm < M) {
-                const float v = __fmul_rn(__uint_as_float(r[i]), alpha);
-                if constexpr (OUT_F32) reinterpret_cast<float*>(p.out)[mm * N + n] = v;
-                else reinterpret_cast<__nv_bfloat16*>(p.out)[mm * N + n] = __float2bfloat16_rn(v);
-              }
+              for (int i = 0; i < 8; ++i) r[0][j * 8 + i] = r8[i];
             }
           }
         }
+        tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(bar_acc_empty);
+        auto store_out = [&](int64_t mm, float v) {
+          if constexpr (OUT_F32) reinterpret_cast<float*>(p.out)[mm * N + n] = v;
+          else reinterpret_cast<__nv_bfloat16*>(p.out)[mm * N + n] = __float2bfloat16_rn(v);
+        };
+        const int64_t tile_u0 = (int64_t)tp * p.kt;
+        const int64_t c_first = cta_of_unit(tile_u0, U, G);
+        const int64_t c_last = cta_of_unit(tile_u0 + p.kt - 1, U, G);
+        if (c_first == c_last) {
+          // the whole K range of this tile ran here
+          if (n < N) {
+#pragma unroll
+            for (int c = 0; c < (BN + 31) / 32; ++c)
+#pragma unroll
+              for (int i = 0; i < kCols; ++i) {
+                const int64_t mm = q0 + c * 32 + i;
+                if (mm < M) store_out(mm, __fmul_rn(__uint_as_float(r[c][i]), alpha));
+              }
+          }
+        } else {
+          // split tile.  The CTA that holds the tile's first K steps (its
+          // last work item, so it finishes last) keeps its partial in
+          // registers, waits for the other contributors' partials -- published
+          // early in their runs -- and adds them in CTA (= K) order.
+          if ((int64_t)blockIdx.x != c_first) {
+            float* part = p.ws + 2 * (int64_t)blockIdx.x * BN * kBM;    // slot of a CTA's first item
+#pragma unroll
+            for (int c = 0; c < (BN + 31) / 32; ++c)
+#pragma unroll
+              for (int i = 0; i < kCols; ++i) {
+                const int mm = c * 32 + i;
+                if (q0 + mm < M) __stcg(part + (int64_t)mm * kBM + row, __uint_as_float(r[c][i]));
+              }
+            named_bar_sync(kEpiBar, 128);      // every partial store of the CTA is issued
+            if (et == 0) {
+              __threadfence();                  // ... and visible GPU-wide before the count
+              atomicAdd(p.tickets + tp, 1);
+            }
+          } else {
+            const int nwait = (int)(c_last - c_first);
+            if (et == 0) {
+              // bounded wait for the other partials of this tile
+              const uint64_t t0 = globaltimer_ns();
+              int ready = 0;
+              while (true) {
+                asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(ready) : "l"(p.tickets + tp) : "memory");
+                if (ready >= nwait) break;
+                if (globaltimer_ns() - t0 > p.timeout_ns) {
+                  atomicCAS(p.err, 0u, kErrTimeout);
+                  break;
+                }
+              }
+              *last_flag = ready >= nwait;
+              p.tickets[tp] = 0;                // ready for the next launch
+            }
+            named_bar_sync(kEpiBar, 128);
+            float sum[(BN + 31) / 32][kCols];
+#pragma unroll
+            for (int cb = 0; cb < (BN + 31) / 32; ++cb)
+#pragma unroll
+              for (int i = 0; i < kCols; ++i) sum[cb][i] = __uint_as_float(r[cb][i]);
+            for (int64_t c = c_first + 1; c <= c_last; ++c) {
+              const float* src = p.ws + 2 * c * (int64_t)BN * kBM + row;
+              float v[(BN + 31) / 32][kCols];
+#pragma unroll
+              for (int cb = 0; cb < (BN + 31) / 32; ++cb)
+#pragma unroll
+                for (int i = 0; i < kCols; ++i) {
+                  const int mm = cb * 32 + i;
+                  v[cb][i] = q0 + mm < M ? __ldcg(src + (int64_t)mm * kBM) : 0.0f;
+                }
+#pragma unroll
+              for (int cb = 0; cb < (BN + 31) / 32; ++cb)
+#pragma unroll
+                for (int i = 0; i < kCols; ++i) sum[cb][i] = __fadd_rn(sum[cb][i], v[cb][i]);
+            }
+            if (n < N && *last_flag) {
+#pragma unroll
+              for (int cb = 0; cb < (BN + 31) / 32; ++cb)
+#pragma unroll
+                for (int i = 0; i < kCols; ++i) {
+                  const int64_t mm = q0 + cb * 32 + i;
+                  if (mm < M) store_out(mm, __fmul_rn(sum[cb][i], alpha));
+                }
+            }
+            named_bar_sync(kEpiBar, 128);      // last_flag is read before it is rewritten
+          }
+        }
       }
       acc_phase ^= 1;
       acc_buf ^= 1;
+      first_item = false;
     }
     if (tma_store && et == 0) bulk_wait_group<0>();   // stores done before the CTA's smem goes away
   }
@@ -563,6 +748,40 @@ bool make_out_map(CUtensorMap* m, void* base, int64_t M, int64_t N, bool f32) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Swapped (decode) tiles are split over the CTAs along K; partial tiles are
+// exchanged through a workspace the library owns: one per (device, stream),
+// allocated on the first swapped call on that stream, kept until exit.
+constexpr int kMaxTickets = 65536;
+
+struct Workspace {
+  float* ws = nullptr;
+  int* tickets = nullptr;
+};
+
+cudaError_t get_workspace(const DeviceInfo* d, cudaStream_t st, Workspace* out) {
+  static std::mutex mu;
+  static std::map<std::pair<int, cudaStream_t>, Workspace> table;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = table.find({d->device, st});
+  if (it != table.end()) {
+    *out = it->second;
+    return cudaSuccess;
+  }
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) return cudaErrorNotPermitted;
+  Workspace w;
+  const size_t ws_bytes = (size_t)2 * d->sm_count * 128 * kBM * sizeof(float);
+  cudaError_t e = cudaMalloc(&w.ws, ws_bytes);
+  if (e != cudaSuccess) return e;
+  e = cudaMalloc(&w.tickets, kMaxTickets * sizeof(int));
+  if (e != cudaSuccess) return e;
+  e = cudaMemset(w.tickets, 0, kMaxTickets * sizeof(int));
+  if (e != cudaSuccess) return e;
+  table[{d->device, st}] = w;
+  *out = w;
+  return cudaSuccess;
+}
+
 template <int BN, bool SWAP, bool OUT_F32>
 cudaError_t launch(const GemmParams& p, const DeviceInfo* d, cudaStream_t st) {
   using Cf = Cfg<BN, SWAP>;
@@ -573,10 +792,28 @@ cudaError_t launch(const GemmParams& p, const DeviceInfo* d, cudaStream_t st) {
     attr_err[d->device] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmemBytes);
   });
   if (attr_err[d->device] != cudaSuccess) return attr_err[d->device];
-  const int tiles = p.tiles_p * p.tiles_q;
-  const int grid = tiles < d->sm_count ? tiles : d->sm_count;
-  kern<<<grid, kThreads, Cf::kSmemBytes, st>>>(p);
-  return cudaGetLastError();
+  int grid;
+  if (SWAP) {
+    const int64_t units = (int64_t)p.tiles_p * p.kt;
+    grid = (int)(units < d->sm_count ? units : d->sm_count);
+  } else {
+    const int tiles = p.tiles_p * p.tiles_q;
+    grid = tiles < d->sm_count ? tiles : d->sm_count;
+  }
+  // programmatic dependent launch: the kernel may start while the previous
+  // kernel in the stream finishes; it waits (griddepcontrol.wait) before
+  // touching anything that kernel produced
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Cf::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
 float alpha_of(float ga, float gw) { return (float)(1.0 / ((double)ga * (double)gw)); }
@@ -602,7 +839,15 @@ nvfp4_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float ga,
 
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
-  const bool swap = M <= 128;
+  const bool swap = M <= 128 && ceil_div(N, kBM) <= kMaxTickets;
+  if (swap) {
+    Workspace w;
+    const cudaError_t e = get_workspace(d, st, &w);
+    if (e == cudaErrorNotPermitted) return NVFP4_ERR_UNSUPPORTED;
+    if (e != cudaSuccess) return cuda_status(e);
+    p.ws = w.ws;
+    p.tickets = w.tickets;
+  }
   int bn = 256;
   if (swap) bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
   p.rows_p = (int)(swap ? N : M);

@@ -160,6 +160,11 @@ __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ 
                                                        uint8_t* __restrict__ scales, float* amax_out,
                                                        int64_t kc) {
   constexpr int U = 2;
+  // programmatic dependent launch: let the next kernel (the GEMM) start its
+  // prologue and weight loads now, and wait until the previous kernel in the
+  // stream has completed before touching memory it may read or write
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ float rtab[256];
   {
     const uint32_t s = threadIdx.x;
@@ -337,9 +342,17 @@ cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, float g, uint8_
   // CTAs (2048 threads) per SM
   const int threads = 256;
   const int blocks = grid_for(ceil_div(total, 2), threads, d, 8);
-  quantize_kernel<kF32, kTC, kAmax><<<blocks, threads, 0, st>>>(x, real, total, nblk, make_div(nblk), g, codes,
-                                                                scales, amax_out, kc);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(threads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, quantize_kernel<kF32, kTC, kAmax>, x, real, total, nblk, make_div(nblk), g, codes,
+                            scales, amax_out, kc);
 }
 
 }  // namespace

@@ -175,3 +175,29 @@ def test_gemm_partial_last_tile_bf16(M, N, K):
         out16 = gpu_gemm(a_d, as_d, ga, w_d, ws_d, gw, M, N, K, torch.bfloat16)
         assert torch.equal(out16, out32.to(torch.bfloat16))
     assert_gemm_close(out32.cpu().numpy(), ref, f"{M}x{N}x{K}")
+
+
+def test_split_k_decode_deterministic_and_stream_local():
+    # decode shapes split K over the CTAs; partials are summed in a fixed
+    # order, so repeated runs match bitwise, also on two streams at once
+    M, N, K = 8, 4096, 5120
+    (ac, asc, ga), (wc, wsc, gw) = _operands(M, N, K, seed=21)
+    a_d, as_d = to_dev_operand(ac, asc, K)
+    w_d, ws_d = to_dev_operand(wc, wsc, K)
+    ref = gpu_gemm(a_d, as_d, ga, w_d, ws_d, gw, M, N, K, torch.bfloat16)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    outs = []
+    for s in (s1, s2):
+        with torch.cuda.stream(s):   # first call on each stream (sets up its workspace)
+            outs.append(gpu_gemm(a_d, as_d, ga, w_d, ws_d, gw, M, N, K, torch.bfloat16))
+    torch.cuda.synchronize()
+    for _ in range(5):
+        o = []
+        for s in (s1, s2):
+            with torch.cuda.stream(s):
+                o.append(gpu_gemm(a_d, as_d, ga, w_d, ws_d, gw, M, N, K, torch.bfloat16))
+        torch.cuda.synchronize()
+        for t in o:
+            assert torch.equal(t, ref)
+    assert all(torch.equal(t, ref) for t in outs)
+    check_device_error_word()
