@@ -496,6 +496,8 @@ def measure_quant_sweep(torch, nv, synth, dev, args, stream, peaks):
     sweep = {}
     for M in synth.QUANT_SWEEP_M:
         for K in synth.QUANT_SWEEP_K:
+            if args.quant_point and args.quant_point != f"{M}x{K}":
+                continue
             q = QuantSweep(torch, nv, synth, dev, M, K)
             kk = max(3, min(args.steps, 50))
             with torch.cuda.stream(stream):
@@ -518,6 +520,7 @@ def main():
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed decode steps first")
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quant-point", default="", help="MxK: run only this point of the quantize sweep")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
