@@ -155,6 +155,34 @@ NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scale
                         int64_t M, int64_t N, int64_t K, void* out, nvfp4_out_dtype out_dtype,
                         nvfp4_stream_t stream);
 
+/* nvfp4_gemm for decode-sized M that allocates nothing.  The pages have no
+ * counterpart: this is an interface variant, not part of the method.  It
+ * computes exactly what nvfp4_gemm computes for the same arguments (same
+ * kernel, same K split, same summation order), but the K-split partial tiles
+ * and arrival counters live in a fixed scratch array in the library's static
+ * device memory instead of a workspace allocated on first use.  For callers
+ * that must not allocate device memory once running (a serving engine that
+ * plans its memory at start-up and gives the rest to its KV cache; code that
+ * cannot take the implicit synchronisation of an allocation).
+ *   Arguments, layouts and alignment: as nvfp4_gemm.
+ *   Limits (the scratch size): M <= 32, N <= 131072, device with at most 160
+ *   SMs.  Scratch: 5 MiB of partial tiles + 4 KiB of counters per device,
+ *   part of the library's module image.
+ *   The counters must be zero when the kernel starts; the call clears them on
+ *   `stream` (cudaMemsetAsync) before each launch.
+ *   The first call on each device resolves the scratch address (once, with
+ *   that device current); make it before any stream capture begins.
+ *   There is ONE scratch array per device: two calls that can run at the same
+ *   time on one device (different streams, no ordering between them) race
+ *   on it and both results are undefined.  Calls ordered on one stream are
+ *   safe.
+ * Errors: INVALID_ARG, ALIGNMENT (as nvfp4_gemm); UNSUPPORTED (M > 32,
+ * N > 131072, more than 160 SMs, or not sm_100); CUDA. */
+NVFP4_API nvfp4_status nvfp4_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_scales, float a_global_scale,
+                                const uint8_t* w_codes, const uint8_t* w_scales, float w_global_scale,
+                                int64_t M, int64_t N, int64_t K, void* out, nvfp4_out_dtype out_dtype,
+                                nvfp4_stream_t stream);
+
 /* Fused projection: the GEMM above with W the row-wise concatenation of
  * n_seg separately calibrated weights; output columns
  * [seg_offsets[i], seg_offsets[i+1]) are rescaled with

@@ -45,6 +45,7 @@ _lib.nvfp4_amax.argtypes = [_vp, ctypes.c_int, _i64, _i64, _vp, _vp]
 _lib.nvfp4_quantize.argtypes = [_vp, ctypes.c_int, _i64, _i64, _f32, _vp, _vp, ctypes.c_int, _vp, _vp]
 _lib.nvfp4_swizzle_scales.argtypes = [_vp, _i64, _i64, _vp, _vp]
 _lib.nvfp4_gemm.argtypes = [_vp, _vp, _f32, _vp, _vp, _f32, _i64, _i64, _i64, _vp, ctypes.c_int, _vp]
+_lib.nvfp4_gemm_noalloc.argtypes = [_vp, _vp, _f32, _vp, _vp, _f32, _i64, _i64, _i64, _vp, ctypes.c_int, _vp]
 _lib.nvfp4_fused_proj.argtypes = [_vp, _vp, _f32, _vp, _vp, ctypes.POINTER(_i64), ctypes.POINTER(_f32),
                                   ctypes.c_int, _i64, _i64, _vp, ctypes.c_int, _vp]
 _lib.nvfp4_convert_e4m3.argtypes = [_vp, _vp, _i64, _vp]
@@ -146,6 +147,14 @@ def nvfp4_gemm(a_codes, a_scales, a_global_scale, w_codes, w_scales, w_global_sc
     _check("nvfp4_gemm", _lib.nvfp4_gemm(_ptr(a_codes), _ptr(a_scales), float(a_global_scale), _ptr(w_codes),
                                          _ptr(w_scales), float(w_global_scale), M, N, K, _ptr(out),
                                          _out_dtype(out), _stream(out)))
+
+
+def nvfp4_gemm_noalloc(a_codes, a_scales, a_global_scale, w_codes, w_scales, w_global_scale, M, N, K,
+                       out: torch.Tensor) -> None:
+    _check("nvfp4_gemm_noalloc",
+           _lib.nvfp4_gemm_noalloc(_ptr(a_codes), _ptr(a_scales), float(a_global_scale), _ptr(w_codes),
+                                   _ptr(w_scales), float(w_global_scale), M, N, K, _ptr(out), _out_dtype(out),
+                                   _stream(out)))
 
 
 def nvfp4_fused_proj(a_codes, a_scales, a_global_scale, w_codes, w_scales, seg_offsets, seg_global_scales,

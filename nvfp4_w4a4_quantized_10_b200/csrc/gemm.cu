@@ -886,6 +886,92 @@ nvfp4_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float ga,
   return cuda_status(e);
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free decode GEMM (nvfp4_gemm_noalloc).  Same kernel and same
+// work split as the swapped (M <= 128) path of nvfp4_gemm, but its K-split
+// scratch is a fixed array in this module's static device memory instead of
+// the per-stream workspace nvfp4_gemm allocates on first use.  It serves
+// callers that must not allocate device memory after start-up: a serving
+// engine that measures its peak memory once and hands the remainder to its
+// KV cache (a later allocation can fail or eat into that cache), and code
+// that cannot afford the implicit device synchronisation cudaMalloc may
+// perform.
+//
+// Limits (the scratch is sized for them; larger inputs are rejected with
+// NVFP4_ERR_UNSUPPORTED): M <= 32, N <= 131072 (1024 weight tiles), at most
+// 160 SMs.  Scratch: partial tiles, 2 slots x 160 CTAs x (32 x 128) FP32 =
+// 5 MiB, then 1024 int arrival counters (4 KiB).
+constexpr int kNoAllocMaxM = 32;
+constexpr int kNoAllocMaxCtas = 160;
+constexpr int kNoAllocMaxTiles = 1024;
+constexpr size_t kNoAllocPartialBytes = (size_t)2 * kNoAllocMaxCtas * kNoAllocMaxM * kBM * sizeof(float);
+constexpr size_t kNoAllocScratchBytes = kNoAllocPartialBytes + kNoAllocMaxTiles * sizeof(int);
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+struct NoAllocScratch {
+  std::once_flag once;
+  cudaError_t err = cudaSuccess;
+  uint8_t* ptr = nullptr;
+};
+NoAllocScratch g_noalloc[64];
+
+nvfp4_status run_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_scales, float ga, const uint8_t* w_codes,
+                              const uint8_t* w_scales, float gw, int64_t M, int64_t N, int64_t K, void* out,
+                              nvfp4_out_dtype out_dtype, cudaStream_t st) {
+  if (!a_codes || !a_scales || !w_codes || !w_scales || !out) return NVFP4_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 32 || K % 32 != 0) return NVFP4_ERR_INVALID_ARG;
+  if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F32) return NVFP4_ERR_INVALID_ARG;
+  if (!finite_positive(ga) || !finite_positive(gw)) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
+      !aligned16(out))
+    return NVFP4_ERR_ALIGNMENT;
+  if (M > kNoAllocMaxM || ceil_div(N, kBM) > kNoAllocMaxTiles || K > (1ll << 31)) return NVFP4_ERR_UNSUPPORTED;
+  const DeviceInfo* d = device_info();
+  if (!d) return NVFP4_ERR_CUDA;
+  if (d->major != 10 || d->sm_count > kNoAllocMaxCtas || d->device >= 64) return NVFP4_ERR_UNSUPPORTED;
+  // once per device, with that device current (device_info() reads the
+  // current device): the scratch array's address on it
+  NoAllocScratch& sc = g_noalloc[d->device];
+  std::call_once(sc.once, [&] { sc.err = cudaGetSymbolAddress((void**)&sc.ptr, g_noalloc_scratch); });
+  if (sc.err != cudaSuccess || !sc.ptr) return NVFP4_ERR_CUDA;
+
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  const int bn = M <= 16 ? 16 : 32;
+  p.ws = reinterpret_cast<float*>(sc.ptr);
+  p.tickets = reinterpret_cast<int*>(sc.ptr + kNoAllocPartialBytes);
+  p.rows_p = (int)N;
+  p.rows_q = (int)M;
+  p.sf_p = w_scales;
+  p.sf_q = a_scales;
+  if (!make_code_map(&p.tmap_p, w_codes, p.rows_p, K, kBM) || !make_code_map(&p.tmap_q, a_codes, p.rows_q, K, bn))
+    return NVFP4_ERR_CUDA;
+  p.out = out;
+  p.tma_store = 0;
+  p.err = d->err_word;
+  p.timeout_ns = wait_timeout_ns();
+  p.M = M;
+  p.N = N;
+  p.rb_q = (int)ceil_div(p.rows_q, 128);
+  p.kc = (int)ceil_div(K, 64);
+  p.kt = (int)ceil_div(K, 256);
+  p.tiles_p = (int)ceil_div(p.rows_p, kBM);
+  p.tiles_q = 1;
+  p.n_seg = 1;
+  p.seg_end[0] = (int)N;
+  p.seg_alpha[0] = alpha_of(ga, gw);
+  // The arrival counters must be zero when the kernel starts.  The kernel
+  // leaves every counter it used at zero, but a launch whose bounded wait ran
+  // out does not, so they are cleared on the stream before every launch.
+  cudaError_t e = cudaMemsetAsync(p.tickets, 0, (size_t)p.tiles_p * sizeof(int), st);
+  if (e != cudaSuccess) return cuda_status(e);
+  const bool f32 = out_dtype == NVFP4_OUT_F32;
+  if (bn == 16) e = f32 ? launch<16, true, true>(p, d, st) : launch<16, true, false>(p, d, st);
+  else e = f32 ? launch<32, true, true>(p, d, st) : launch<32, true, false>(p, d, st);
+  return cuda_status(e);
+}
+
 }  // namespace
 }  // namespace nvfp4
 
@@ -909,6 +995,13 @@ nvfp4_status nvfp4_fused_proj(const uint8_t* a_codes, const uint8_t* a_scales, f
   if (!seg_offsets || !seg_global_scales || n_seg < 1 || n_seg > NVFP4_MAX_SEGMENTS) return NVFP4_ERR_INVALID_ARG;
   return run_gemm(a_codes, a_scales, a_global_scale, w_codes, w_scales, seg_offsets, seg_global_scales, n_seg, M,
                   seg_offsets[n_seg], K, out, out_dtype, (cudaStream_t)stream);
+}
+
+nvfp4_status nvfp4_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_scales, float a_global_scale,
+                                const uint8_t* w_codes, const uint8_t* w_scales, float w_global_scale, int64_t M,
+                                int64_t N, int64_t K, void* out, nvfp4_out_dtype out_dtype, nvfp4_stream_t stream) {
+  return run_gemm_noalloc(a_codes, a_scales, a_global_scale, w_codes, w_scales, w_global_scale, M, N, K, out,
+                          out_dtype, (cudaStream_t)stream);
 }
 
 }  // extern "C"
