@@ -47,7 +47,6 @@ namespace nvfp4 {
 constexpr int kBM = 128;          // MMA M: rows of operand P per tile
 constexpr int kBKBytes = 128;     // bytes of codes per row per stage (256 elements)
 constexpr int kSfChunk = 512;     // bytes of one 128-row x 4-scale chunk
-constexpr int kThreads = 192;
 constexpr int kTmemCols = 512;
 constexpr int kGroupP = 8;        // tile raster: 8 P-tiles share a Q-tile
 constexpr int kStageOutBytes = 16384;   // one 128-row x 128-byte output sub-tile
@@ -94,7 +93,15 @@ struct Cfg {
   static constexpr int kOffSfb = kOffSfa + kStages * kSfaBytes;
   static constexpr int kOffOut = kOffSfb + kStages * kSfbBytes;      // 1024-aligned
   static constexpr int kOffBar = kOffOut + kOutBytes;
-  static constexpr int kNumBars = 2 * kStages + 3;                   // full, empty, acc_full, acc_empty, drain
+  // Swapped tiles: two extra warps issue the scale copies (warp 6: P's
+  // scales, warp 7: Q's) so that the MMA warp issues only MMAs; a tcgen05
+  // instruction holds its issuing thread for tens of cycles, but instructions
+  // from different threads proceed in parallel.
+  static constexpr bool kSplitCopy = SWAP;
+  static constexpr int kThreads = kSplitCopy ? 256 : 192;
+  // full, empty, acc_full, acc_empty, drain; with split copies also one
+  // scales-ready barrier per stage and one drain barrier per copy warp
+  static constexpr int kNumBars = 2 * kStages + 3 + (kSplitCopy ? kStages + 2 : 0);
   static constexpr int kOffSeg = kOffBar + kNumBars * 8;             // segment table: ends, alphas
   static constexpr int kOffMisc = kOffSeg + 2 * 4 * NVFP4_MAX_SEGMENTS;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;            // + alignment slack
@@ -202,7 +209,7 @@ __device__ __forceinline__ float seg_alpha_smem(const int* ends, const float* al
 __device__ __forceinline__ uint32_t swz128(uint32_t r, uint32_t c) { return r * 128 + ((c ^ (r & 7)) << 4); }
 
 template <int BN, bool SWAP, bool OUT_F32>
-__global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(const __grid_constant__ GemmParams p) {
   using C = Cfg<BN, SWAP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -212,6 +219,8 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
   const uint32_t bar_acc_full = bar_empty + 8 * C::kStages;
   const uint32_t bar_acc_empty = bar_acc_full + 8;
   const uint32_t bar_drain = bar_acc_empty + 8;
+  const uint32_t bar_sf = bar_drain + 8;                     // [kStages], split copies only
+  const uint32_t bar_cp_drain = bar_sf + 8 * C::kStages;     // [2], split copies only
   int* seg_end_s = reinterpret_cast<int*>(smem + C::kOffSeg);
   float* seg_alpha_s = reinterpret_cast<float*>(smem + C::kOffSeg + 4 * NVFP4_MAX_SEGMENTS);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
@@ -232,6 +241,11 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
     mbar_init(bar_acc_full, 1);
     mbar_init(bar_acc_empty, 128);
     mbar_init(bar_drain, 1);
+    if (C::kSplitCopy) {
+      for (int s = 0; s < C::kStages; ++s) mbar_init(bar_sf + 8 * s, 2);
+      mbar_init(bar_cp_drain, 1);
+      mbar_init(bar_cp_drain + 8, 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&p.tmap_p);
@@ -253,10 +267,12 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    // The weight operand (P when swapped, Q otherwise) does not depend on
-    // the preceding kernel, so the weight side of the first kStages steps is
-    // requested before waiting on it (programmatic dependent launch); every
-    // activation load comes after griddepcontrol.wait.
+    // Programmatic dependent launch: this kernel may start while the
+    // preceding kernel in the stream still runs, and that kernel may be
+    // writing any of the inputs (the weight included).  Before
+    // griddepcontrol.wait the weight tiles of the first kStages steps are
+    // only prefetched into L2 (a hint that reads nothing into the CTA); every
+    // load into shared memory comes after the wait.
     if (lane == 0) {
       const int kc = p.kc, rb_q = p.rb_q;
       uint32_t issued_mask = 0, last_parity = 0;   // for the drain on abort
@@ -300,16 +316,21 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
       // prologue: the first kStages stages are free
       int npro = 0;
       for_steps(w0, 0, C::kStages, [&](int j, int p0, int q0, int k) {
-        expect(j, q0, k);
-        if (SWAP) load_p(j, p0, k);
-        else load_q(j, q0, k);
-        issued_mask |= 1u << j;
+        const uint32_t sf_bytes = (uint32_t)min(4, kc - 4 * k) * kSfChunk;
+        if (SWAP) {
+          tma_prefetch_l2_2d(&p.tmap_p, k * kBKBytes, p0);
+          bulk_prefetch_l2(p.sf_p + ((size_t)(p0 >> 7) * kc + 4 * k) * kSfChunk, sf_bytes);
+        } else {
+          tma_prefetch_l2_2d(&p.tmap_q, k * kBKBytes, q0);
+        }
         npro = j + 1;
       });
       asm volatile("griddepcontrol.wait;" ::: "memory");
       for_steps(w0, 0, npro, [&](int j, int p0, int q0, int k) {
-        if (SWAP) load_q(j, q0, k);
-        else load_p(j, p0, k);
+        expect(j, q0, k);
+        load_p(j, p0, k);
+        load_q(j, q0, k);
+        issued_mask |= 1u << j;
       });
       int stage = npro % C::kStages;
       uint32_t phase = npro == C::kStages ? 1u : 0u;
@@ -355,6 +376,33 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
       tc_fence_after();
       const uint32_t acc = tmem_base + (acc_buf ? C::kAcc1Col : 0);
       for (int k = kb0; k < ke0; ++k) {
+        if (C::kSplitCopy) {
+          // the copy warps waited for the stage's data and moved its scales
+          if (!mbar_wait(bar_sf + 8 * stage, phase, abort_flag, p.err, p.timeout_ns)) { ok = false; break; }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t sfa_t = sf_t0 + stage * C::kSfStageCols;
+            const uint32_t sfb_t = sfa_t + C::kSfaCols;
+            const uint64_t ad = a_desc0 + (uint64_t)((stage * C::kABytes) >> 4);
+            const uint64_t bd = b_desc0 + (uint64_t)((stage * C::kBBytes) >> 4);
+            const uint32_t acc_in = k != kb0 ? 1u : 0u;
+            const int nkb = min(4, kc - 4 * k);
+            if (nkb == 4) {
+#pragma unroll
+              for (int kb = 0; kb < 4; ++kb)
+                tc_mma_nvf4(acc, ad + (uint64_t)(kb * 2), bd + (uint64_t)(kb * 2), idesc, sfa_t + kb * 4,
+                            sfb_t + kb * 4 * C::kSfbBlocks, (acc_in | kb) != 0 ? 1u : 0u);
+            } else {
+              for (int kb = 0; kb < nkb; ++kb)
+                tc_mma_nvf4(acc, ad + (uint64_t)(kb * 2), bd + (uint64_t)(kb * 2), idesc, sfa_t + kb * 4,
+                            sfb_t + kb * 4 * C::kSfbBlocks, (acc_in | kb) != 0 ? 1u : 0u);
+            }
+            tc_commit(bar_empty + 8 * stage);
+          }
+          __syncwarp();
+          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+          continue;
+        }
         if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, p.err, p.timeout_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t sb = sbase + C::kOffSfb + stage * C::kSfbBytes;
@@ -411,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
       (void)mbar_wait(bar_drain, 0, &never, p.err, p.timeout_ns);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 6) {
     // ------------------------------------------------------------ epilogue
     const int sp = warp & 3;                 // TMEM subpartition of this warp
     const int row = sp * 32 + lane;          // accumulator lane = tile row of P
@@ -687,6 +735,55 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_gemm_kernel(const __grid_co
       first_item = false;
     }
     if (tma_store && et == 0) bulk_wait_group<0>();   // stores done before the CTA's smem goes away
+  } else if (C::kSplitCopy) {
+    // ------------------------------------------------------------ scale copies
+    // warp 6 copies P's scale chunks of each stage into TMEM, warp 7 Q's; each
+    // then commits to the stage's scales-ready barrier (2 arrivals).  The
+    // TMEM scale region of a stage is rewritten only after the stage's next
+    // full barrier, i.e. after the producer saw the MMAs that read it finish.
+    const bool copy_p = warp == 6;
+    if (lane == 0) {
+      const uint64_t desc0 = smem_desc(sbase + (copy_p ? C::kOffSfa : C::kOffSfb), 16, 128, 0);
+      const uint32_t sf_t0 = tmem_base + C::kSfBase;
+      const int kc = p.kc;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      WorkIter w = work_begin(p, SWAP);
+      int tp, tq, kb0, ke0;
+      while (ok && work_next(p, w, tp, tq, kb0, ke0)) {
+        for (int k = kb0; k < ke0; ++k) {
+          if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, p.err, p.timeout_ns)) { ok = false; break; }
+          const uint32_t sfa_t = sf_t0 + stage * C::kSfStageCols;
+          const int nkb = min(4, kc - 4 * k);
+          if (copy_p) {
+            const uint64_t d = desc0 + (uint64_t)((stage * C::kSfaBytes) >> 4);
+            if (nkb == 4) {
+#pragma unroll
+              for (int kb = 0; kb < 4; ++kb) tc_cp_32x128b_warpx4(sfa_t + kb * 4, d + (uint64_t)(kb * (kSfChunk >> 4)));
+            } else {
+              for (int kb = 0; kb < nkb; ++kb) tc_cp_32x128b_warpx4(sfa_t + kb * 4, d + (uint64_t)(kb * (kSfChunk >> 4)));
+            }
+          } else {
+            const uint64_t d = desc0 + (uint64_t)((stage * C::kSfbBytes) >> 4);
+            const uint32_t sfb_t = sfa_t + C::kSfaCols;
+            for (int kb = 0; kb < nkb; ++kb)
+#pragma unroll
+              for (int rb = 0; rb < C::kSfbBlocks; ++rb)
+                tc_cp_32x128b_warpx4(sfb_t + kb * 4 * C::kSfbBlocks + rb * 4,
+                                     d + (uint64_t)((rb * 4 + kb) * (kSfChunk >> 4)));
+          }
+          tc_commit(bar_sf + 8 * stage);
+          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+        }
+      }
+      // every copy issued by this thread has landed before TMEM is freed
+      const uint32_t db = bar_cp_drain + (copy_p ? 0 : 8);
+      tc_commit(db);
+      volatile int never = 0;
+      (void)mbar_wait(db, 0, &never, p.err, p.timeout_ns);
+    }
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -805,7 +902,7 @@ cudaError_t launch(const GemmParams& p, const DeviceInfo* d, cudaStream_t st) {
   // touching anything that kernel produced
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(Cf::kThreads);
   cfg.dynamicSmemBytes = Cf::kSmemBytes;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];

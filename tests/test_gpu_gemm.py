@@ -201,3 +201,28 @@ def test_split_k_decode_deterministic_and_stream_local():
             assert torch.equal(t, ref)
     assert all(torch.equal(t, ref) for t in outs)
     check_device_error_word()
+
+
+@pytest.mark.parametrize("M,N,K", [(32, 4096, 17408), (8, 12288, 5120), (512, 2048, 5120)])
+def test_gemm_right_after_the_kernel_that_writes_its_operands(M, N, K):
+    # the weight and the activation are quantized on the GPU by the kernels
+    # just before the GEMM on the same stream, with no synchronization: the
+    # GEMM may start early (programmatic dependent launch) but must not read
+    # either operand before those kernels have finished
+    a = synth.student_t_outliers(M, K, seed=M + 1, dtype=torch.float32)
+    w = synth.normal((N, K), seed=N + 2, std=0.02)
+    ac, asc, ga = oracle_quantize(a.numpy())
+    wc, wsc, gw = oracle_quantize(w.numpy())
+    ref = oracle.gemm(ac, asc, ga, wc, wsc, gw)
+    a_d = a.to(DEV)
+    w_d = w.to(DEV)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        wcd, wsd, _ = gpu_quantize(w_d, gw)
+        acd, asd, _ = gpu_quantize(a_d, ga)
+        out = torch.empty(M, N, dtype=torch.float32, device=DEV)
+        nv.nvfp4_gemm(acd, asd, float(ga), wcd, wsd, float(gw), M, N, K, out)
+        torch.cuda.synchronize()
+        assert_gemm_close(out.cpu().numpy(), ref, f"{M}x{N}x{K}")
+        del wcd, wsd, acd, asd
+    check_device_error_word()
