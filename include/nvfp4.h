@@ -143,11 +143,11 @@ NVFP4_API nvfp4_status nvfp4_swizzle_scales(const uint8_t* rowmajor, int64_t row
  * fixed order (the result does not depend on timing and equals the unsplit
  * sum up to FP32 rounding order).  The partials go to a workspace the
  * library allocates on first use for each (device, stream) pair
- * (2 * SMs * 64 KB plus 256 KB of counters) and keeps until the process
- * exits.  That first call on a stream must not be made while the stream is
- * being captured into a CUDA graph: it returns UNSUPPORTED then.  Calls on
- * one stream share its workspace safely (stream order); calls on different
- * streams use different workspaces.
+ * (2 * SMs * 128 KB) and keeps until the process exits.  That first call on a
+ * stream must not be made while the stream is being captured into a CUDA
+ * graph: it returns UNSUPPORTED then.  Calls on one stream share its
+ * workspace safely (stream order); calls on different streams use different
+ * workspaces.
  * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (device is not sm_100, or a
  * first decode-shaped call during capture), CUDA. */
 NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float a_global_scale,
@@ -165,19 +165,20 @@ NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scale
  * plans its memory at start-up and gives the rest to its KV cache; code that
  * cannot take the implicit synchronisation of an allocation).
  *   Arguments, layouts and alignment: as nvfp4_gemm.
- *   Limits (the scratch size): M <= 32, N <= 131072, device with at most 160
- *   SMs.  Scratch: 5 MiB of partial tiles + 4 KiB of counters per device,
- *   part of the library's module image.
- *   The counters must be zero when the kernel starts; the call clears them on
- *   `stream` (cudaMemsetAsync) before each launch.
+ *   Limits (the scratch size): M <= 32, device with at most 160 SMs.
+ *   Scratch: 10 MiB of tagged partial-tile words per device, part of the
+ *   library's module image.  Every word must be empty (zero) when a launch
+ *   starts: the array is zeroed when the module loads, every launch leaves
+ *   the words it used empty, and nvfp4_last_device_error() empties it after
+ *   a launch that reported an error.
  *   The first call on each device resolves the scratch address (once, with
  *   that device current); make it before any stream capture begins.
  *   There is ONE scratch array per device: two calls that can run at the same
  *   time on one device (different streams, no ordering between them) race
  *   on it and both results are undefined.  Calls ordered on one stream are
  *   safe.
- * Errors: INVALID_ARG, ALIGNMENT (as nvfp4_gemm); UNSUPPORTED (M > 32,
- * N > 131072, more than 160 SMs, or not sm_100); CUDA. */
+ * Errors: INVALID_ARG, ALIGNMENT (as nvfp4_gemm); UNSUPPORTED (M > 32, more
+ * than 160 SMs, or not sm_100); CUDA. */
 NVFP4_API nvfp4_status nvfp4_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_scales, float a_global_scale,
                                 const uint8_t* w_codes, const uint8_t* w_scales, float w_global_scale,
                                 int64_t M, int64_t N, int64_t K, void* out, nvfp4_out_dtype out_dtype,
@@ -210,7 +211,10 @@ NVFP4_API nvfp4_status nvfp4_convert_e4m3(const float* in, uint8_t* out, int64_t
 NVFP4_API nvfp4_status nvfp4_convert_e2m1(const float* in, uint8_t* out, int64_t n, nvfp4_stream_t stream);
 
 /* Synchronizes the current device, then returns and clears its device error
- * word: NVFP4_OK, NVFP4_ERR_TIMEOUT or NVFP4_ERR_DEVICE. */
+ * word: NVFP4_OK, NVFP4_ERR_TIMEOUT or NVFP4_ERR_DEVICE.  When the word was
+ * set it also empties the GEMM's K-split scratch on this device (a launch that
+ * gave up may leave partial tiles behind); GEMM results after a reported
+ * error are reliable only once this call has returned. */
 NVFP4_API nvfp4_status nvfp4_last_device_error(void);
 
 /* Bound (nanoseconds) on every wait inside this library's kernels on all

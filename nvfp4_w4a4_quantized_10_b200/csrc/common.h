@@ -26,6 +26,10 @@ const DeviceInfo* device_info();
 // Wait bound for every kernel of the library (ns).
 uint64_t wait_timeout_ns();
 
+// Empties every K-split scratch buffer of the GEMM on `device` (after a
+// device-side error left partial words behind).  Synchronous.
+cudaError_t clear_gemm_scratch(int device);
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline bool finite_positive(float g) {

@@ -59,8 +59,7 @@ struct alignas(64) GemmParams {
   const uint8_t* sf_p;
   const uint8_t* sf_q;
   void* out;
-  float* ws;             // swapped tiles: FP32 partial tiles, 2 slots per CTA
-  int* tickets;          // swapped tiles: per-tile arrival counters (zero between launches)
+  uint64_t* ws;          // swapped tiles: tagged FP32 partial tiles, 2 slots per CTA (all words empty between launches)
   unsigned* err;
   uint64_t timeout_ns;
   int64_t M, N;          // output [M, N]
@@ -204,6 +203,28 @@ __device__ __forceinline__ float seg_alpha_smem(const int* ends, const float* al
   return alphas[seg_index_smem(ends, n_seg, n)];
 }
 
+// Tagged partial words: FP32 bits in the low half, kFullTag in the high half
+// once written; 0 = empty.  An aligned 64-bit store or load is single-copy
+// atomic, so a reader that sees the tag sees the value.
+constexpr uint32_t kFullTag = 1u;
+
+__device__ __forceinline__ void st_full_word(uint64_t* p, uint32_t value_bits) {
+  const uint64_t w = ((uint64_t)kFullTag << 32) | value_bits;
+  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+
+__device__ __forceinline__ void st_word(uint64_t* p, uint64_t w) {
+  asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+
+// No "memory" clobber: the polls of one round are independent and may all be
+// in flight together (volatile keeps each round's loads inside its loop).
+__device__ __forceinline__ uint64_t ld_word(const uint64_t* p) {
+  uint64_t w;
+  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(w) : "l"(p));
+  return w;
+}
+
 // Byte offset of 16-byte chunk c of row r in a 128-row x 128-byte sub-tile
 // stored with the 128B swizzle the output tensor map uses.
 __device__ __forceinline__ uint32_t swz128(uint32_t r, uint32_t c) { return r * 128 + ((c ^ (r & 7)) << 4); }
@@ -225,7 +246,6 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
   float* seg_alpha_s = reinterpret_cast<float*>(smem + C::kOffSeg + 4 * NVFP4_MAX_SEGMENTS);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
-  volatile int* last_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -661,63 +681,66 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
               }
           }
         } else {
-          // split tile.  The CTA that holds the tile's first K steps (its
-          // last work item, so it finishes last) keeps its partial in
-          // registers, waits for the other contributors' partials -- published
-          // early in their runs -- and adds them in CTA (= K) order.
+          // split tile.  The CTA that holds the tile's first K steps (its last
+          // work item, so it finishes last) adds the tile up in CTA (= K)
+          // order, its own partial from registers.  Every other contributor
+          // writes its partial to its slot (2c for CTA c's first item, 2c + 1
+          // for its last) as 64-bit words that carry the FP32 value in the low
+          // half and a "full" tag in the high half: one single-copy-atomic
+          // store per value, so no fence or counter is needed.  The adder
+          // polls each word until it is full and clears it for the next
+          // launch.
           if ((int64_t)blockIdx.x != c_first) {
-            float* part = p.ws + 2 * (int64_t)blockIdx.x * BN * kBM;    // slot of a CTA's first item
+            uint64_t* part = p.ws + (2 * (int64_t)blockIdx.x + (first_item ? 0 : 1)) * BN * kBM + row;
 #pragma unroll
             for (int c = 0; c < (BN + 31) / 32; ++c)
 #pragma unroll
               for (int i = 0; i < kCols; ++i) {
                 const int mm = c * 32 + i;
-                if (q0 + mm < M) __stcg(part + (int64_t)mm * kBM + row, __uint_as_float(r[c][i]));
+                if (q0 + mm < M) st_full_word(part + (int64_t)mm * kBM, r[c][i]);
               }
-            named_bar_sync(kEpiBar, 128);      // every partial store of the CTA is issued
-            if (et == 0) {
-              __threadfence();                  // ... and visible GPU-wide before the count
-              atomicAdd(p.tickets + tp, 1);
-            }
           } else {
-            const int nwait = (int)(c_last - c_first);
-            if (et == 0) {
-              // bounded wait for the other partials of this tile
-              const uint64_t t0 = globaltimer_ns();
-              int ready = 0;
-              while (true) {
-                asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(ready) : "l"(p.tickets + tp) : "memory");
-                if (ready >= nwait) break;
-                if (globaltimer_ns() - t0 > p.timeout_ns) {
-                  atomicCAS(p.err, 0u, kErrTimeout);
-                  break;
-                }
-              }
-              *last_flag = ready >= nwait;
-              p.tickets[tp] = 0;                // ready for the next launch
-            }
-            named_bar_sync(kEpiBar, 128);
             float sum[(BN + 31) / 32][kCols];
 #pragma unroll
             for (int cb = 0; cb < (BN + 31) / 32; ++cb)
 #pragma unroll
               for (int i = 0; i < kCols; ++i) sum[cb][i] = __uint_as_float(r[cb][i]);
+            bool ok_all = true;
             for (int64_t c = c_first + 1; c <= c_last; ++c) {
-              const float* src = p.ws + 2 * c * (int64_t)BN * kBM + row;
-              float v[(BN + 31) / 32][kCols];
+              const int64_t slot = 2 * c + (unit_begin(c, U, G) >= tile_u0 ? 0 : 1);
+              uint64_t* src = p.ws + slot * BN * kBM + row;
+              uint64_t v[(BN + 31) / 32][kCols];
+              const uint64_t t0 = globaltimer_ns();
+              while (true) {
+#pragma unroll
+                for (int cb = 0; cb < (BN + 31) / 32; ++cb)
+#pragma unroll
+                  for (int i = 0; i < kCols; ++i) {
+                    const int mm = cb * 32 + i;
+                    v[cb][i] = q0 + mm < M ? ld_word(src + (int64_t)mm * kBM) : (uint64_t)kFullTag << 32;
+                  }
+                uint32_t all = 1;
+#pragma unroll
+                for (int cb = 0; cb < (BN + 31) / 32; ++cb)
+#pragma unroll
+                  for (int i = 0; i < kCols; ++i) all &= (uint32_t)((v[cb][i] >> 32) == kFullTag);
+                if (all) break;
+                if (globaltimer_ns() - t0 > p.timeout_ns) {
+                  atomicCAS(p.err, 0u, kErrTimeout);
+                  ok_all = false;
+                  break;
+                }
+              }
 #pragma unroll
               for (int cb = 0; cb < (BN + 31) / 32; ++cb)
 #pragma unroll
                 for (int i = 0; i < kCols; ++i) {
                   const int mm = cb * 32 + i;
-                  v[cb][i] = q0 + mm < M ? __ldcg(src + (int64_t)mm * kBM) : 0.0f;
+                  sum[cb][i] = __fadd_rn(sum[cb][i], __uint_as_float((uint32_t)v[cb][i]));
+                  if (q0 + mm < M) st_word(src + (int64_t)mm * kBM, 0ull);     // empty again
                 }
-#pragma unroll
-              for (int cb = 0; cb < (BN + 31) / 32; ++cb)
-#pragma unroll
-                for (int i = 0; i < kCols; ++i) sum[cb][i] = __fadd_rn(sum[cb][i], v[cb][i]);
             }
-            if (n < N && *last_flag) {
+            if (n < N && ok_all) {
 #pragma unroll
               for (int cb = 0; cb < (BN + 31) / 32; ++cb)
 #pragma unroll
@@ -726,7 +749,6 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
                   if (mm < M) store_out(mm, __fmul_rn(sum[cb][i], alpha));
                 }
             }
-            named_bar_sync(kEpiBar, 128);      // last_flag is read before it is rewritten
           }
         }
       }
@@ -847,34 +869,32 @@ bool make_out_map(CUtensorMap* m, void* base, int64_t M, int64_t N, bool f32) {
 
 // Swapped (decode) tiles are split over the CTAs along K; partial tiles are
 // exchanged through a workspace the library owns: one per (device, stream),
-// allocated on the first swapped call on that stream, kept until exit.
-constexpr int kMaxTickets = 65536;
-
+// allocated (all words empty) on the first swapped call on that stream, kept
+// until exit.
 struct Workspace {
-  float* ws = nullptr;
-  int* tickets = nullptr;
+  uint64_t* ws = nullptr;
+  size_t bytes = 0;
 };
 
+std::mutex g_ws_mu;
+std::map<std::pair<int, cudaStream_t>, Workspace> g_ws_table;
+
 cudaError_t get_workspace(const DeviceInfo* d, cudaStream_t st, Workspace* out) {
-  static std::mutex mu;
-  static std::map<std::pair<int, cudaStream_t>, Workspace> table;
-  std::lock_guard<std::mutex> lock(mu);
-  auto it = table.find({d->device, st});
-  if (it != table.end()) {
+  std::lock_guard<std::mutex> lock(g_ws_mu);
+  auto it = g_ws_table.find({d->device, st});
+  if (it != g_ws_table.end()) {
     *out = it->second;
     return cudaSuccess;
   }
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
   if (cudaStreamIsCapturing(st, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) return cudaErrorNotPermitted;
   Workspace w;
-  const size_t ws_bytes = (size_t)2 * d->sm_count * 128 * kBM * sizeof(float);
-  cudaError_t e = cudaMalloc(&w.ws, ws_bytes);
+  w.bytes = (size_t)2 * d->sm_count * 128 * kBM * sizeof(uint64_t);
+  cudaError_t e = cudaMalloc(&w.ws, w.bytes);
   if (e != cudaSuccess) return e;
-  e = cudaMalloc(&w.tickets, kMaxTickets * sizeof(int));
+  e = cudaMemset(w.ws, 0, w.bytes);
   if (e != cudaSuccess) return e;
-  e = cudaMemset(w.tickets, 0, kMaxTickets * sizeof(int));
-  if (e != cudaSuccess) return e;
-  table[{d->device, st}] = w;
+  g_ws_table[{d->device, st}] = w;
   *out = w;
   return cudaSuccess;
 }
@@ -936,14 +956,13 @@ nvfp4_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float ga,
 
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
-  const bool swap = M <= 128 && ceil_div(N, kBM) <= kMaxTickets;
+  const bool swap = M <= 128;
   if (swap) {
     Workspace w;
     const cudaError_t e = get_workspace(d, st, &w);
     if (e == cudaErrorNotPermitted) return NVFP4_ERR_UNSUPPORTED;
     if (e != cudaSuccess) return cuda_status(e);
     p.ws = w.ws;
-    p.tickets = w.tickets;
   }
   int bn = 256;
   if (swap) bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
@@ -995,14 +1014,14 @@ nvfp4_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float ga,
 // perform.
 //
 // Limits (the scratch is sized for them; larger inputs are rejected with
-// NVFP4_ERR_UNSUPPORTED): M <= 32, N <= 131072 (1024 weight tiles), at most
-// 160 SMs.  Scratch: partial tiles, 2 slots x 160 CTAs x (32 x 128) FP32 =
-// 5 MiB, then 1024 int arrival counters (4 KiB).
+// NVFP4_ERR_UNSUPPORTED): M <= 32, at most 160 SMs.  Scratch: tagged partial
+// tiles, 2 slots x 160 CTAs x (32 x 128) 64-bit words = 10 MiB.  Every word
+// must be empty (zero) when a launch starts: the array is zero-initialised
+// when the module loads, each launch leaves every word it used empty, and
+// after a launch that timed out nvfp4_last_device_error() clears it.
 constexpr int kNoAllocMaxM = 32;
 constexpr int kNoAllocMaxCtas = 160;
-constexpr int kNoAllocMaxTiles = 1024;
-constexpr size_t kNoAllocPartialBytes = (size_t)2 * kNoAllocMaxCtas * kNoAllocMaxM * kBM * sizeof(float);
-constexpr size_t kNoAllocScratchBytes = kNoAllocPartialBytes + kNoAllocMaxTiles * sizeof(int);
+constexpr size_t kNoAllocScratchBytes = (size_t)2 * kNoAllocMaxCtas * kNoAllocMaxM * kBM * sizeof(uint64_t);
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
@@ -1012,6 +1031,31 @@ struct NoAllocScratch {
   uint8_t* ptr = nullptr;
 };
 NoAllocScratch g_noalloc[64];
+
+}  // namespace
+
+// After a launch whose bounded wait ran out, partial words may be left full;
+// empty every K-split scratch of the current device (library workspaces and
+// the allocation-free scratch).  Synchronous.
+cudaError_t clear_gemm_scratch(int device) {
+  cudaError_t first = cudaSuccess;
+  {
+    std::lock_guard<std::mutex> lock(g_ws_mu);
+    for (auto& kv : g_ws_table)
+      if (kv.first.first == device) {
+        const cudaError_t e = cudaMemset(kv.second.ws, 0, kv.second.bytes);
+        if (first == cudaSuccess) first = e;
+      }
+  }
+  if (device >= 0 && device < 64 && g_noalloc[device].ptr) {
+    const cudaError_t e = cudaMemset(g_noalloc[device].ptr, 0, kNoAllocScratchBytes);
+    if (first == cudaSuccess) first = e;
+  }
+  const cudaError_t e = cudaDeviceSynchronize();
+  return first == cudaSuccess ? e : first;
+}
+
+namespace {
 
 nvfp4_status run_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_scales, float ga, const uint8_t* w_codes,
                               const uint8_t* w_scales, float gw, int64_t M, int64_t N, int64_t K, void* out,
@@ -1023,7 +1067,7 @@ nvfp4_status run_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_scales, f
   if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
       !aligned16(out))
     return NVFP4_ERR_ALIGNMENT;
-  if (M > kNoAllocMaxM || ceil_div(N, kBM) > kNoAllocMaxTiles || K > (1ll << 31)) return NVFP4_ERR_UNSUPPORTED;
+  if (M > kNoAllocMaxM || N > (1ll << 31) - 256 || K > (1ll << 31)) return NVFP4_ERR_UNSUPPORTED;
   const DeviceInfo* d = device_info();
   if (!d) return NVFP4_ERR_CUDA;
   if (d->major != 10 || d->sm_count > kNoAllocMaxCtas || d->device >= 64) return NVFP4_ERR_UNSUPPORTED;
@@ -1036,8 +1080,7 @@ nvfp4_status run_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_scales, f
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
   const int bn = M <= 16 ? 16 : 32;
-  p.ws = reinterpret_cast<float*>(sc.ptr);
-  p.tickets = reinterpret_cast<int*>(sc.ptr + kNoAllocPartialBytes);
+  p.ws = reinterpret_cast<uint64_t*>(sc.ptr);
   p.rows_p = (int)N;
   p.rows_q = (int)M;
   p.sf_p = w_scales;
@@ -1058,11 +1101,7 @@ nvfp4_status run_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_scales, f
   p.n_seg = 1;
   p.seg_end[0] = (int)N;
   p.seg_alpha[0] = alpha_of(ga, gw);
-  // The arrival counters must be zero when the kernel starts.  The kernel
-  // leaves every counter it used at zero, but a launch whose bounded wait ran
-  // out does not, so they are cleared on the stream before every launch.
-  cudaError_t e = cudaMemsetAsync(p.tickets, 0, (size_t)p.tiles_p * sizeof(int), st);
-  if (e != cudaSuccess) return cuda_status(e);
+  cudaError_t e;
   const bool f32 = out_dtype == NVFP4_OUT_F32;
   if (bn == 16) e = f32 ? launch<16, true, true>(p, d, st) : launch<16, true, false>(p, d, st);
   else e = f32 ? launch<32, true, true>(p, d, st) : launch<32, true, false>(p, d, st);

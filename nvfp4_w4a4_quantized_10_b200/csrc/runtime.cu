@@ -90,6 +90,7 @@ nvfp4_status nvfp4_last_device_error(void) {
   const unsigned zero = 0;
   if (cudaMemcpy(d->err_word, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
     return NVFP4_ERR_CUDA;
+  if (w != 0 && clear_gemm_scratch(d->device) != cudaSuccess) return NVFP4_ERR_CUDA;
   if (w == kErrTimeout) return NVFP4_ERR_TIMEOUT;
   if (w != 0) return NVFP4_ERR_DEVICE;
   return NVFP4_OK;

@@ -28,3 +28,25 @@ def test_wait_timeout_setting_round_trips():
     gpu_quantize(x, 50.0)
     torch.cuda.synchronize()
     assert nv.nvfp4_last_device_error() == nv.OK
+
+
+def test_error_read_back_clears_gemm_scratch_and_gemm_still_agrees():
+    # reading back a device error also empties the decode GEMM's K-split
+    # scratch (library workspaces and the allocation-free array); GEMMs on
+    # both paths must give the same result before and after
+    M, N, K = 8, 4096, 5120
+    x = torch.randn(M, K, device=DEV).to(torch.bfloat16)
+    w = (0.02 * torch.randn(N, K, device=DEV)).to(torch.bfloat16)
+    ac, asc, _ = gpu_quantize(x, 300.0)
+    wc, wsc, _ = gpu_quantize(w, 20000.0)
+    outs = []
+    for _ in range(2):
+        o1 = torch.empty(M, N, dtype=torch.float32, device=DEV)
+        o2 = torch.empty(M, N, dtype=torch.float32, device=DEV)
+        nv.nvfp4_gemm(ac, asc, 300.0, wc, wsc, 20000.0, M, N, K, o1)
+        nv.nvfp4_gemm_noalloc(ac, asc, 300.0, wc, wsc, 20000.0, M, N, K, o2)
+        assert nv.nvfp4_last_device_error() == nv.OK
+        outs += [o1, o2]
+        nv.nvfp4_test_wait_timeout(1_000_000, DEV)
+        assert nv.nvfp4_last_device_error() == nv.ERR_TIMEOUT
+    assert all(torch.equal(o, outs[0]) for o in outs[1:])
