@@ -92,33 +92,42 @@ struct Cfg {
   static constexpr int kOffSfb = kOffSfa + kStages * kSfaBytes;
   static constexpr int kOffOut = kOffSfb + kStages * kSfbBytes;      // 1024-aligned
   static constexpr int kOffBar = kOffOut + kOutBytes;
-  // Swapped tiles: two extra warps issue the scale copies (warp 6: P's
-  // scales, warp 7: Q's) so that the MMA warp issues only MMAs; a tcgen05
-  // instruction holds its issuing thread for tens of cycles, but instructions
-  // from different threads proceed in parallel.
-  static constexpr bool kSplitCopy = SWAP;
-  static constexpr int kThreads = kSplitCopy ? 256 : 192;
+  // Two extra warps issue the scale copies (warp 6: P's scales, warp 7: Q's)
+  // so that the MMA warp issues only MMAs; a tcgen05 instruction holds its
+  // issuing thread for tens of cycles, but instructions from different
+  // threads proceed in parallel.
+#ifndef NVFP4_SPLIT_COPY_NORMAL
+#define NVFP4_SPLIT_COPY_NORMAL 1
+#endif
+  static constexpr bool kSplitCopy = SWAP || NVFP4_SPLIT_COPY_NORMAL;
+  // one copy warp for P's scales and one per 128-row block of Q's
+  static constexpr int kCopyWarps = kSplitCopy ? 1 + kSfbBlocks : 0;
+  static constexpr int kThreads = 192 + 32 * kCopyWarps;
   // full, empty, acc_full, acc_empty, drain; with split copies also one
   // scales-ready barrier per stage and one drain barrier per copy warp
-  static constexpr int kNumBars = 2 * kStages + 3 + (kSplitCopy ? kStages + 2 : 0);
+  static constexpr int kNumBars = 2 * kStages + 3 + (kSplitCopy ? kStages + kCopyWarps : 0);
   static constexpr int kOffSeg = kOffBar + kNumBars * 8;             // segment table: ends, alphas
   static constexpr int kOffMisc = kOffSeg + 2 * 4 * NVFP4_MAX_SEGMENTS;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;            // + alignment slack
-  // TMEM columns.  Normal 128x256 tiles: two accumulator buffers, [0,256)
-  // and [192,448), overlapping in 64 columns, so tile t+1 can start as soon
-  // as the epilogue has drained the 64 shared columns of tile t; the scale
-  // factors of the stage being computed sit in [448,496) (tcgen05 operations
-  // of one thread execute in issue order, so one scale region serves every
-  // stage).  Swapped (decode) tiles: one accumulator and one scale region per
-  // pipeline stage.
+  // TMEM columns.  Normal 128x256 tiles: two accumulator buffers that
+  // overlap, so tile t+1 can start as soon as the epilogue has drained the
+  // shared columns of tile t (the epilogue drains those first).  With split
+  // copies the copy warps run ahead of the MMAs, so the scales need a ring of
+  // regions: two regions of 48 columns at [416,512), accumulators [0,256) and
+  // [160,416) sharing 96 columns.  With one issuing thread, tcgen05
+  // operations execute in issue order and one region at [448,496) serves
+  // every stage: accumulators [0,256) and [192,448) share 64 columns.
+  // Swapped (decode) tiles: one accumulator and one scale region per pipeline
+  // stage.
   static constexpr int kAccCols = BN < 32 ? 32 : BN;
   static constexpr bool kOverlapAcc = !SWAP && BN == 256;
-  static constexpr int kAcc1Col = kOverlapAcc ? 192 : 0;
+  static constexpr int kAcc1Col = kOverlapAcc ? (kSplitCopy ? 160 : 192) : 0;
+  static constexpr int kSharedSlots = kOverlapAcc ? (kSplitCopy ? 2 : 1) : 0;   // 64-column slots drained before release
   static constexpr int kSfaCols = 16;                                // 4 MMAs x 4 columns
   static constexpr int kSfbCols = kSfbBlocks * 16;
   static constexpr int kSfStageCols = kSfaCols + kSfbCols;
-  static constexpr int kSfBase = kOverlapAcc ? 448 : kAccCols;
-  static constexpr int kSfRegions = kOverlapAcc ? 1 : kStages;
+  static constexpr int kSfBase = kOverlapAcc ? (kSplitCopy ? 416 : 448) : kAccCols;
+  static constexpr int kSfRegions = kOverlapAcc ? (kSplitCopy ? 2 : 1) : kStages;
   static_assert(kStages >= 2, "pipeline depth");
   static_assert(kSfBase + kSfRegions * kSfStageCols <= kTmemCols, "TMEM budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -241,7 +250,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
   const uint32_t bar_acc_empty = bar_acc_full + 8;
   const uint32_t bar_drain = bar_acc_empty + 8;
   const uint32_t bar_sf = bar_drain + 8;                     // [kStages], split copies only
-  const uint32_t bar_cp_drain = bar_sf + 8 * C::kStages;     // [2], split copies only
+  const uint32_t bar_cp_drain = bar_sf + 8 * C::kStages;     // [kCopyWarps], split copies only
   int* seg_end_s = reinterpret_cast<int*>(smem + C::kOffSeg);
   float* seg_alpha_s = reinterpret_cast<float*>(smem + C::kOffSeg + 4 * NVFP4_MAX_SEGMENTS);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
@@ -262,9 +271,8 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
     mbar_init(bar_acc_empty, 128);
     mbar_init(bar_drain, 1);
     if (C::kSplitCopy) {
-      for (int s = 0; s < C::kStages; ++s) mbar_init(bar_sf + 8 * s, 2);
-      mbar_init(bar_cp_drain, 1);
-      mbar_init(bar_cp_drain + 8, 1);
+      for (int s = 0; s < C::kStages; ++s) mbar_init(bar_sf + 8 * s, C::kCopyWarps);
+      for (int i = 0; i < C::kCopyWarps; ++i) mbar_init(bar_cp_drain + 8 * i, 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -386,7 +394,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
     const uint64_t sfb_desc0 = smem_desc(sbase + C::kOffSfb, 16, 128, 0);
     const uint32_t sf_t0 = tmem_base + C::kSfBase;
     const int kc = p.kc;
-    int stage = 0;
+    int stage = 0, region = 0;
     uint32_t phase = 0, acc_phase = 0, acc_buf = 0;
     bool ok = true;
     WorkIter w = work_begin(p, SWAP);
@@ -401,7 +409,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
           if (!mbar_wait(bar_sf + 8 * stage, phase, abort_flag, p.err, p.timeout_ns)) { ok = false; break; }
           tc_fence_after();
           if (lane == 0) {
-            const uint32_t sfa_t = sf_t0 + stage * C::kSfStageCols;
+            const uint32_t sfa_t = sf_t0 + region * C::kSfStageCols;
             const uint32_t sfb_t = sfa_t + C::kSfaCols;
             const uint64_t ad = a_desc0 + (uint64_t)((stage * C::kABytes) >> 4);
             const uint64_t bd = b_desc0 + (uint64_t)((stage * C::kBBytes) >> 4);
@@ -421,6 +429,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
           }
           __syncwarp();
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+          if (++region == C::kSfRegions) region = 0;
           continue;
         }
         if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, p.err, p.timeout_ns)) { ok = false; break; }
@@ -506,7 +515,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
         // shares with the other one; TMEM is handed back right after them.
         const uint32_t tacc = taddr + (acc_buf ? C::kAcc1Col : 0);
         auto slot_col = [&](int slot) -> int {
-          return C::kOverlapAcc && acc_buf == 0 ? ((slot + 3) & 3) * 64 : slot * 64;
+          return C::kOverlapAcc && acc_buf == 0 ? ((slot + 4 - C::kSharedSlots) & 3) * 64 : slot * 64;
         };
         if constexpr (!OUT_F32) {
           // drain the whole accumulator row into registers (bf16 pairs)
@@ -518,7 +527,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
             tmem_ld_32x32b_x32(tacc + col, r0);
             tmem_ld_32x32b_x32(tacc + col + 32, r1);
             tmem_ld_wait();
-            if (slot == 0 && C::kOverlapAcc) {
+            if (slot == C::kSharedSlots - 1 && C::kOverlapAcc) {
               tc_fence_before();
               mbar_arrive(bar_acc_empty);
             }
@@ -599,7 +608,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
             __syncwarp();
             tmem_ld_32x32b_x32(tacc + c * 32, r);
             tmem_ld_wait();
-            if (cc == 1 && C::kOverlapAcc) {
+            if (cc == 2 * C::kSharedSlots - 1 && C::kOverlapAcc) {
               tc_fence_before();
               mbar_arrive(bar_acc_empty);
             }
@@ -759,16 +768,18 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
     if (tma_store && et == 0) bulk_wait_group<0>();   // stores done before the CTA's smem goes away
   } else if (C::kSplitCopy) {
     // ------------------------------------------------------------ scale copies
-    // warp 6 copies P's scale chunks of each stage into TMEM, warp 7 Q's; each
-    // then commits to the stage's scales-ready barrier (2 arrivals).  The
-    // TMEM scale region of a stage is rewritten only after the stage's next
-    // full barrier, i.e. after the producer saw the MMAs that read it finish.
+    // warp 6 copies P's scale chunks of each stage into TMEM, warp 7 + rb the
+    // chunks of Q's 128-row block rb; each then commits to the stage's
+    // scales-ready barrier (kCopyWarps arrivals).  A TMEM scale region is
+    // rewritten only once the MMAs that read it last have completed.
     const bool copy_p = warp == 6;
+    const int rbq = warp - 7;                   // Q block of this warp
     if (lane == 0) {
       const uint64_t desc0 = smem_desc(sbase + (copy_p ? C::kOffSfa : C::kOffSfb), 16, 128, 0);
       const uint32_t sf_t0 = tmem_base + C::kSfBase;
       const int kc = p.kc;
-      int stage = 0;
+      int stage = 0, region = 0;
+      int64_t step = 0;                         // pipeline steps issued so far
       uint32_t phase = 0;
       bool ok = true;
       WorkIter w = work_begin(p, SWAP);
@@ -776,7 +787,16 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
       while (ok && work_next(p, w, tp, tq, kb0, ke0)) {
         for (int k = kb0; k < ke0; ++k) {
           if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, p.err, p.timeout_ns)) { ok = false; break; }
-          const uint32_t sfa_t = sf_t0 + stage * C::kSfStageCols;
+          if (C::kSfRegions < C::kStages && step >= C::kSfRegions) {
+            // the MMAs of step - kSfRegions read this region: wait for their
+            // commit on that step's empty barrier (the full barrier above
+            // already covers steps at least kStages back)
+            const int64_t s2 = step - C::kSfRegions;
+            if (!mbar_wait(bar_empty + 8 * (int)(s2 % C::kStages), (uint32_t)((s2 / C::kStages) & 1), abort_flag, p.err,
+                           p.timeout_ns)) { ok = false; break; }
+            tc_fence_after();
+          }
+          const uint32_t sfa_t = sf_t0 + region * C::kSfStageCols;
           const int nkb = min(4, kc - 4 * k);
           if (copy_p) {
             const uint64_t d = desc0 + (uint64_t)((stage * C::kSfaBytes) >> 4);
@@ -790,17 +810,17 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
             const uint64_t d = desc0 + (uint64_t)((stage * C::kSfbBytes) >> 4);
             const uint32_t sfb_t = sfa_t + C::kSfaCols;
             for (int kb = 0; kb < nkb; ++kb)
-#pragma unroll
-              for (int rb = 0; rb < C::kSfbBlocks; ++rb)
-                tc_cp_32x128b_warpx4(sfb_t + kb * 4 * C::kSfbBlocks + rb * 4,
-                                     d + (uint64_t)((rb * 4 + kb) * (kSfChunk >> 4)));
+              tc_cp_32x128b_warpx4(sfb_t + kb * 4 * C::kSfbBlocks + rbq * 4,
+                                   d + (uint64_t)((rbq * 4 + kb) * (kSfChunk >> 4)));
           }
           tc_commit(bar_sf + 8 * stage);
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+          if (++region == C::kSfRegions) region = 0;
+          ++step;
         }
       }
       // every copy issued by this thread has landed before TMEM is freed
-      const uint32_t db = bar_cp_drain + (copy_p ? 0 : 8);
+      const uint32_t db = bar_cp_drain + 8 * (warp - 6);
       tc_commit(db);
       volatile int never = 0;
       (void)mbar_wait(db, 0, &never, p.err, p.timeout_ns);
