@@ -496,7 +496,6 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
     const uint32_t taddr = tmem_base + ((uint32_t)(sp * 32) << 16);
     const int64_t M = p.M, N = p.N;
     const int n_seg = p.n_seg;
-    const float alpha0 = seg_alpha_s[0];
     const bool tma_store = !SWAP && p.tma_store;
     uint32_t acc_phase = 0, acc_buf = 0;
     uint32_t out_buf = 0;                    // next staging buffer (TMA store path)
@@ -532,13 +531,21 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
               mbar_arrive(bar_acc_empty);
             }
             const int64_t n0 = q0 + col;
-            if (n_seg == 1) {
+            // one scale for the whole 64-column slot unless a segment
+            // boundary falls inside it
+            int seg_lo = 0, seg_hi = 0;
+            if (n_seg > 1) {
+              seg_lo = seg_index_smem(seg_end_s, n_seg, n0);
+              seg_hi = seg_index_smem(seg_end_s, n_seg, n0 + 63 < N ? n0 + 63 : N - 1);
+            }
+            if (seg_lo == seg_hi) {
+              const float a = seg_alpha_s[seg_lo];
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
-                packed[slot * 32 + i] = pack_bf16x2(__fmul_rn(__uint_as_float(r0[2 * i]), alpha0),
-                                                    __fmul_rn(__uint_as_float(r0[2 * i + 1]), alpha0));
-                packed[slot * 32 + 16 + i] = pack_bf16x2(__fmul_rn(__uint_as_float(r1[2 * i]), alpha0),
-                                                         __fmul_rn(__uint_as_float(r1[2 * i + 1]), alpha0));
+                packed[slot * 32 + i] = pack_bf16x2(__fmul_rn(__uint_as_float(r0[2 * i]), a),
+                                                    __fmul_rn(__uint_as_float(r0[2 * i + 1]), a));
+                packed[slot * 32 + 16 + i] = pack_bf16x2(__fmul_rn(__uint_as_float(r1[2 * i]), a),
+                                                         __fmul_rn(__uint_as_float(r1[2 * i + 1]), a));
               }
             } else {
 #pragma unroll
@@ -612,10 +619,22 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
               tc_fence_before();
               mbar_arrive(bar_acc_empty);
             }
+            const int64_t n0 = q0 + c * 32;
+            int seg_lo = 0, seg_hi = 0;
+            if (n_seg > 1) {
+              seg_lo = seg_index_smem(seg_end_s, n_seg, n0);
+              seg_hi = seg_index_smem(seg_end_s, n_seg, n0 + 31 < N ? n0 + 31 : N - 1);
+            }
+            if (seg_lo == seg_hi) {
+              const float a = seg_alpha_s[seg_lo];
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              r[i] = __float_as_uint(
-                  __fmul_rn(__uint_as_float(r[i]), seg_alpha_smem(seg_end_s, seg_alpha_s, n_seg, q0 + c * 32 + i)));
+              for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__fmul_rn(__uint_as_float(r[i]), a));
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                r[i] = __float_as_uint(
+                    __fmul_rn(__uint_as_float(r[i]), seg_alpha_smem(seg_end_s, seg_alpha_s, n_seg, n0 + i)));
+            }
             if (tma_store && q0 + c * 32 < N) {
               const uint32_t buf = sbase + C::kOffOut + out_buf * kStageOutBytes;
               if (et == 0) bulk_wait_group_read<1>();
