@@ -45,7 +45,6 @@
 namespace nvfp4 {
 
 constexpr int kBM = 128;          // MMA M: rows of operand P per tile
-constexpr int kBKBytes = 128;     // bytes of codes per row per stage (256 elements)
 constexpr int kSfChunk = 512;     // bytes of one 128-row x 4-scale chunk
 constexpr int kTmemCols = 512;
 constexpr int kGroupP = 8;        // tile raster: 8 P-tiles share a Q-tile
@@ -66,7 +65,7 @@ struct alignas(64) GemmParams {
   int rows_p, rows_q;    // rows of the P and Q operands
   int rb_q;              // 128-row scale blocks allocated for Q
   int kc;                // ceil(K / 64): scale chunks per row block
-  int kt;                // ceil(K / 256): pipeline steps per tile
+  int kt;                // ceil(K / (64 * kKB)): pipeline steps per tile
   int tiles_p, tiles_q;
   int tma_store;         // 1: output through shared memory and TMA stores
   int n_seg;
@@ -76,14 +75,23 @@ struct alignas(64) GemmParams {
 
 template <int BN, bool SWAP>
 struct Cfg {
+  // K per pipeline step: kKB blocks of 64 (one MMA each), 256 deep, as
+  // 128-byte rows with the 128B swizzle.  (128-deep steps with 64-byte rows
+  // and the 64B swizzle also work, and fit twice as many stages, but measured
+  // 40 % slower on prefill tiles: the per-step barrier and commit work then
+  // outweighs the earlier buffer release.)
+  static constexpr int kKB = 4;
+  static constexpr int kRowBytes = 32 * kKB;                         // code bytes per row per step
+  static constexpr uint32_t kSwizzleLayout = kRowBytes == 128 ? 2u : 4u;   // descriptor layout type
+  static constexpr uint32_t kSbo = 8 * kRowBytes;                    // bytes between 8-row groups
   static constexpr int kSfbBlocks = (BN + 127) / 128;                // 128-row scale blocks of Q
-  static constexpr int kABytes = kBM * kBKBytes;                     // 16 KB
-  static constexpr int kBBytes = BN * kBKBytes;
-  static constexpr int kSfaBytes = 4 * kSfChunk;                     // 2 KB
-  static constexpr int kSfbBytes = kSfbBlocks * 4 * kSfChunk;
+  static constexpr int kABytes = kBM * kRowBytes;
+  static constexpr int kBBytes = BN * kRowBytes;
+  static constexpr int kSfaBytes = kKB * kSfChunk;
+  static constexpr int kSfbBytes = kSfbBlocks * kKB * kSfChunk;
   static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
   static constexpr int kOutBytes = SWAP ? 0 : 2 * kStageOutBytes;    // double-buffered output sub-tiles
-  static constexpr int kMaxStages = SWAP ? 8 : 4;
+  static constexpr int kMaxStages = 8;
   static constexpr int kFit = (222 * 1024 - kOutBytes) / kStageBytes;
   static constexpr int kStages = kFit < kMaxStages ? kFit : kMaxStages;
   static constexpr int kOffA = 0;
@@ -92,42 +100,36 @@ struct Cfg {
   static constexpr int kOffSfb = kOffSfa + kStages * kSfaBytes;
   static constexpr int kOffOut = kOffSfb + kStages * kSfbBytes;      // 1024-aligned
   static constexpr int kOffBar = kOffOut + kOutBytes;
-  // Two extra warps issue the scale copies (warp 6: P's scales, warp 7: Q's)
-  // so that the MMA warp issues only MMAs; a tcgen05 instruction holds its
-  // issuing thread for tens of cycles, but instructions from different
-  // threads proceed in parallel.
-#ifndef NVFP4_SPLIT_COPY_NORMAL
-#define NVFP4_SPLIT_COPY_NORMAL 1
-#endif
-  static constexpr bool kSplitCopy = SWAP || NVFP4_SPLIT_COPY_NORMAL;
-  // one copy warp for P's scales and one per 128-row block of Q's
-  static constexpr int kCopyWarps = kSplitCopy ? 1 + kSfbBlocks : 0;
+  // Extra warps issue the scale copies (warp 6: P's scales, warp 7 + rb: the
+  // scales of Q's 128-row block rb) so that the MMA warp issues only MMAs; a
+  // tcgen05 instruction holds its issuing thread for tens of cycles, but
+  // instructions from different threads proceed in parallel.
+  static constexpr int kCopyWarps = 1 + kSfbBlocks;
   static constexpr int kThreads = 192 + 32 * kCopyWarps;
-  // full, empty, acc_full, acc_empty, drain; with split copies also one
-  // scales-ready barrier per stage and one drain barrier per copy warp
-  static constexpr int kNumBars = 2 * kStages + 3 + (kSplitCopy ? kStages + kCopyWarps : 0);
+  // full, empty, acc_full, acc_empty, drain, one scales-ready barrier per
+  // stage and one drain barrier per copy warp
+  static constexpr int kNumBars = 2 * kStages + 3 + kStages + kCopyWarps;
   static constexpr int kOffSeg = kOffBar + kNumBars * 8;             // segment table: ends, alphas
   static constexpr int kOffMisc = kOffSeg + 2 * 4 * NVFP4_MAX_SEGMENTS;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;            // + alignment slack
-  // TMEM columns.  Normal 128x256 tiles: two accumulator buffers that
+  // TMEM columns.  Normal 128x256 tiles: the copy warps run ahead of the
+  // MMAs, so the scales of successive steps use a ring of two regions at the
+  // top of TMEM ([416,512) for 48-column regions); the two accumulator
+  // buffers, [0,256) and [kAcc1Col, kAcc1Col + 256), fill the rest and
   // overlap, so tile t+1 can start as soon as the epilogue has drained the
-  // shared columns of tile t (the epilogue drains those first).  With split
-  // copies the copy warps run ahead of the MMAs, so the scales need a ring of
-  // regions: two regions of 48 columns at [416,512), accumulators [0,256) and
-  // [160,416) sharing 96 columns.  With one issuing thread, tcgen05
-  // operations execute in issue order and one region at [448,496) serves
-  // every stage: accumulators [0,256) and [192,448) share 64 columns.
-  // Swapped (decode) tiles: one accumulator and one scale region per pipeline
-  // stage.
+  // shared columns of tile t (it drains those 64-column slots first).
+  // Swapped (decode) tiles: one accumulator and one scale region per
+  // pipeline stage.
   static constexpr int kAccCols = BN < 32 ? 32 : BN;
   static constexpr bool kOverlapAcc = !SWAP && BN == 256;
-  static constexpr int kAcc1Col = kOverlapAcc ? (kSplitCopy ? 160 : 192) : 0;
-  static constexpr int kSharedSlots = kOverlapAcc ? (kSplitCopy ? 2 : 1) : 0;   // 64-column slots drained before release
-  static constexpr int kSfaCols = 16;                                // 4 MMAs x 4 columns
-  static constexpr int kSfbCols = kSfbBlocks * 16;
+  static constexpr int kSfaCols = 4 * kKB;                           // kKB MMAs x 4 columns
+  static constexpr int kSfbCols = kSfbBlocks * 4 * kKB;
   static constexpr int kSfStageCols = kSfaCols + kSfbCols;
-  static constexpr int kSfBase = kOverlapAcc ? (kSplitCopy ? 416 : 448) : kAccCols;
-  static constexpr int kSfRegions = kOverlapAcc ? (kSplitCopy ? 2 : 1) : kStages;
+  static constexpr int kSfRegions = kOverlapAcc ? 2 : kStages;
+  static constexpr int kSfBase = kOverlapAcc ? kTmemCols - kSfRegions * kSfStageCols : kAccCols;
+  static constexpr int kAcc1Col = kOverlapAcc ? kSfBase - 256 : 0;
+  static constexpr int kSharedSlots = kOverlapAcc ? (256 - kAcc1Col + 63) / 64 : 0;   // drained before release
+  static_assert(kAcc1Col % 32 == 0, "accumulator column alignment");
   static_assert(kStages >= 2, "pipeline depth");
   static_assert(kSfBase + kSfRegions * kSfStageCols <= kTmemCols, "TMEM budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -249,8 +251,8 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
   const uint32_t bar_acc_full = bar_empty + 8 * C::kStages;
   const uint32_t bar_acc_empty = bar_acc_full + 8;
   const uint32_t bar_drain = bar_acc_empty + 8;
-  const uint32_t bar_sf = bar_drain + 8;                     // [kStages], split copies only
-  const uint32_t bar_cp_drain = bar_sf + 8 * C::kStages;     // [kCopyWarps], split copies only
+  const uint32_t bar_sf = bar_drain + 8;                     // [kStages]
+  const uint32_t bar_cp_drain = bar_sf + 8 * C::kStages;     // [kCopyWarps]
   int* seg_end_s = reinterpret_cast<int*>(smem + C::kOffSeg);
   float* seg_alpha_s = reinterpret_cast<float*>(smem + C::kOffSeg + 4 * NVFP4_MAX_SEGMENTS);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
@@ -270,10 +272,8 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
     mbar_init(bar_acc_full, 1);
     mbar_init(bar_acc_empty, 128);
     mbar_init(bar_drain, 1);
-    if (C::kSplitCopy) {
-      for (int s = 0; s < C::kStages; ++s) mbar_init(bar_sf + 8 * s, C::kCopyWarps);
-      for (int i = 0; i < C::kCopyWarps; ++i) mbar_init(bar_cp_drain + 8 * i, 1);
-    }
+    for (int s = 0; s < C::kStages; ++s) mbar_init(bar_sf + 8 * s, C::kCopyWarps);
+    for (int i = 0; i < C::kCopyWarps; ++i) mbar_init(bar_cp_drain + 8 * i, 1);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&p.tmap_p);
@@ -320,36 +320,36 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
       };
       auto load_p = [&](int stage, int p0, int k) {
         const uint32_t fb = bar_full + 8 * stage;
-        const uint32_t sf_bytes = (uint32_t)min(4, kc - 4 * k) * kSfChunk;
-        tma_load_2d(sbase + C::kOffA + stage * C::kABytes, &p.tmap_p, k * kBKBytes, p0, fb);
+        const uint32_t sf_bytes = (uint32_t)min(C::kKB, kc - C::kKB * k) * kSfChunk;
+        tma_load_2d(sbase + C::kOffA + stage * C::kABytes, &p.tmap_p, k * C::kRowBytes, p0, fb);
         bulk_load(sbase + C::kOffSfa + stage * C::kSfaBytes,
-                  p.sf_p + ((size_t)(p0 >> 7) * kc + 4 * k) * kSfChunk, sf_bytes, fb);
+                  p.sf_p + ((size_t)(p0 >> 7) * kc + C::kKB * k) * kSfChunk, sf_bytes, fb);
       };
       auto load_q = [&](int stage, int q0, int k) {
         const uint32_t fb = bar_full + 8 * stage;
-        const uint32_t sf_bytes = (uint32_t)min(4, kc - 4 * k) * kSfChunk;
+        const uint32_t sf_bytes = (uint32_t)min(C::kKB, kc - C::kKB * k) * kSfChunk;
         const int nsfb = nsfb_of(q0);
-        tma_load_2d(sbase + C::kOffB + stage * C::kBBytes, &p.tmap_q, k * kBKBytes, q0, fb);
+        tma_load_2d(sbase + C::kOffB + stage * C::kBBytes, &p.tmap_q, k * C::kRowBytes, q0, fb);
 #pragma unroll
         for (int rb = 0; rb < C::kSfbBlocks; ++rb)
           if (rb < nsfb)
-            bulk_load(sbase + C::kOffSfb + stage * C::kSfbBytes + rb * 4 * kSfChunk,
-                      p.sf_q + ((size_t)((q0 >> 7) + rb) * kc + 4 * k) * kSfChunk, sf_bytes, fb);
+            bulk_load(sbase + C::kOffSfb + stage * C::kSfbBytes + rb * C::kKB * kSfChunk,
+                      p.sf_q + ((size_t)((q0 >> 7) + rb) * kc + C::kKB * k) * kSfChunk, sf_bytes, fb);
       };
       auto expect = [&](int stage, int q0, int k) {
-        const uint32_t sf_bytes = (uint32_t)min(4, kc - 4 * k) * kSfChunk;
+        const uint32_t sf_bytes = (uint32_t)min(C::kKB, kc - C::kKB * k) * kSfChunk;
         mbar_arrive_expect_tx(bar_full + 8 * stage, C::kABytes + C::kBBytes + sf_bytes * (1 + nsfb_of(q0)));
       };
       const WorkIter w0 = work_begin(p, SWAP);
       // prologue: the first kStages stages are free
       int npro = 0;
       for_steps(w0, 0, C::kStages, [&](int j, int p0, int q0, int k) {
-        const uint32_t sf_bytes = (uint32_t)min(4, kc - 4 * k) * kSfChunk;
+        const uint32_t sf_bytes = (uint32_t)min(C::kKB, kc - C::kKB * k) * kSfChunk;
         if (SWAP) {
-          tma_prefetch_l2_2d(&p.tmap_p, k * kBKBytes, p0);
-          bulk_prefetch_l2(p.sf_p + ((size_t)(p0 >> 7) * kc + 4 * k) * kSfChunk, sf_bytes);
+          tma_prefetch_l2_2d(&p.tmap_p, k * C::kRowBytes, p0);
+          bulk_prefetch_l2(p.sf_p + ((size_t)(p0 >> 7) * kc + C::kKB * k) * kSfChunk, sf_bytes);
         } else {
-          tma_prefetch_l2_2d(&p.tmap_q, k * kBKBytes, q0);
+          tma_prefetch_l2_2d(&p.tmap_q, k * C::kRowBytes, q0);
         }
         npro = j + 1;
       });
@@ -384,14 +384,13 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // The whole warp follows the pipeline; lane 0 issues every tcgen05 operation.
+    // The whole warp follows the pipeline; lane 0 issues every MMA.  The copy
+    // warps waited for each stage's data and moved its scales into TMEM.
     constexpr uint32_t idesc = idesc_nvf4(kBM, BN);
     // Descriptors of stage 0, k-block 0; later stages and k-blocks only move
     // the 14-bit start-address field (address >> 4), which never carries.
-    const uint64_t a_desc0 = smem_desc(sbase + C::kOffA, 16, 1024, 2);
-    const uint64_t b_desc0 = smem_desc(sbase + C::kOffB, 16, 1024, 2);
-    const uint64_t sfa_desc0 = smem_desc(sbase + C::kOffSfa, 16, 128, 0);
-    const uint64_t sfb_desc0 = smem_desc(sbase + C::kOffSfb, 16, 128, 0);
+    const uint64_t a_desc0 = smem_desc(sbase + C::kOffA, 16, C::kSbo, C::kSwizzleLayout);
+    const uint64_t b_desc0 = smem_desc(sbase + C::kOffB, 16, C::kSbo, C::kSwizzleLayout);
     const uint32_t sf_t0 = tmem_base + C::kSfBase;
     const int kc = p.kc;
     int stage = 0, region = 0;
@@ -404,75 +403,30 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
       tc_fence_after();
       const uint32_t acc = tmem_base + (acc_buf ? C::kAcc1Col : 0);
       for (int k = kb0; k < ke0; ++k) {
-        if (C::kSplitCopy) {
-          // the copy warps waited for the stage's data and moved its scales
-          if (!mbar_wait(bar_sf + 8 * stage, phase, abort_flag, p.err, p.timeout_ns)) { ok = false; break; }
-          tc_fence_after();
-          if (lane == 0) {
-            const uint32_t sfa_t = sf_t0 + region * C::kSfStageCols;
-            const uint32_t sfb_t = sfa_t + C::kSfaCols;
-            const uint64_t ad = a_desc0 + (uint64_t)((stage * C::kABytes) >> 4);
-            const uint64_t bd = b_desc0 + (uint64_t)((stage * C::kBBytes) >> 4);
-            const uint32_t acc_in = k != kb0 ? 1u : 0u;
-            const int nkb = min(4, kc - 4 * k);
-            if (nkb == 4) {
-#pragma unroll
-              for (int kb = 0; kb < 4; ++kb)
-                tc_mma_nvf4(acc, ad + (uint64_t)(kb * 2), bd + (uint64_t)(kb * 2), idesc, sfa_t + kb * 4,
-                            sfb_t + kb * 4 * C::kSfbBlocks, (acc_in | kb) != 0 ? 1u : 0u);
-            } else {
-              for (int kb = 0; kb < nkb; ++kb)
-                tc_mma_nvf4(acc, ad + (uint64_t)(kb * 2), bd + (uint64_t)(kb * 2), idesc, sfa_t + kb * 4,
-                            sfb_t + kb * 4 * C::kSfbBlocks, (acc_in | kb) != 0 ? 1u : 0u);
-            }
-            tc_commit(bar_empty + 8 * stage);
-          }
-          __syncwarp();
-          if (++stage == C::kStages) { stage = 0; phase ^= 1; }
-          if (++region == C::kSfRegions) region = 0;
-          continue;
-        }
-        if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, p.err, p.timeout_ns)) { ok = false; break; }
+        if (!mbar_wait(bar_sf + 8 * stage, phase, abort_flag, p.err, p.timeout_ns)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t sb = sbase + C::kOffSfb + stage * C::kSfbBytes;
         if (lane == 0) {
-          const uint32_t sfa_t = sf_t0 + (C::kSfRegions == 1 ? 0 : stage) * C::kSfStageCols;
+          const uint32_t sfa_t = sf_t0 + region * C::kSfStageCols;
           const uint32_t sfb_t = sfa_t + C::kSfaCols;
           const uint64_t ad = a_desc0 + (uint64_t)((stage * C::kABytes) >> 4);
           const uint64_t bd = b_desc0 + (uint64_t)((stage * C::kBBytes) >> 4);
-          const uint64_t sad = sfa_desc0 + (uint64_t)((stage * C::kSfaBytes) >> 4);
-          const uint64_t sbd = sfb_desc0 + (uint64_t)((stage * C::kSfbBytes) >> 4);
           const uint32_t acc_in = k != kb0 ? 1u : 0u;
-          // TMEM column of Q's scales for K-block kb (multiples of 4 columns)
-          auto sfq_col = [&](int kb, int rb) -> uint32_t { return sfb_t + kb * 4 * C::kSfbBlocks + rb * 4; };
-          if (4 * k + 4 <= kc) {
+          const int nkb = min(C::kKB, kc - C::kKB * k);
+          if (nkb == C::kKB) {
 #pragma unroll
-            for (int kb = 0; kb < 4; ++kb) {
-              tc_cp_32x128b_warpx4(sfa_t + kb * 4, sad + (uint64_t)(kb * (kSfChunk >> 4)));
-#pragma unroll
-              for (int rb = 0; rb < C::kSfbBlocks; ++rb)
-                tc_cp_32x128b_warpx4(sfq_col(kb, rb), sbd + (uint64_t)((rb * 4 + kb) * (kSfChunk >> 4)));
-            }
-#pragma unroll
-            for (int kb = 0; kb < 4; ++kb)
+            for (int kb = 0; kb < C::kKB; ++kb)
               tc_mma_nvf4(acc, ad + (uint64_t)(kb * 2), bd + (uint64_t)(kb * 2), idesc, sfa_t + kb * 4,
-                          sfq_col(kb, 0), (acc_in | kb) != 0 ? 1u : 0u);
+                          sfb_t + kb * 4 * C::kSfbBlocks, (acc_in | kb) != 0 ? 1u : 0u);
           } else {
-            const int nkb = kc - 4 * k;
-            for (int kb = 0; kb < nkb; ++kb) {
-              tc_cp_32x128b_warpx4(sfa_t + kb * 4, sad + (uint64_t)(kb * (kSfChunk >> 4)));
-#pragma unroll
-              for (int rb = 0; rb < C::kSfbBlocks; ++rb)
-                tc_cp_32x128b_warpx4(sfq_col(kb, rb), sbd + (uint64_t)((rb * 4 + kb) * (kSfChunk >> 4)));
-            }
             for (int kb = 0; kb < nkb; ++kb)
               tc_mma_nvf4(acc, ad + (uint64_t)(kb * 2), bd + (uint64_t)(kb * 2), idesc, sfa_t + kb * 4,
-                          sfq_col(kb, 0), (acc_in | kb) != 0 ? 1u : 0u);
+                          sfb_t + kb * 4 * C::kSfbBlocks, (acc_in | kb) != 0 ? 1u : 0u);
           }
           tc_commit(bar_empty + 8 * stage);
         }
         __syncwarp();
         if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+        if (++region == C::kSfRegions) region = 0;
       }
       if (!ok) break;
       if (lane == 0) tc_commit(bar_acc_full);
@@ -734,39 +688,38 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
 #pragma unroll
               for (int i = 0; i < kCols; ++i) sum[cb][i] = __uint_as_float(r[cb][i]);
             bool ok_all = true;
-            for (int64_t c = c_first + 1; c <= c_last; ++c) {
+            for (int64_t c = c_first + 1; c <= c_last && ok_all; ++c) {
               const int64_t slot = 2 * c + (unit_begin(c, U, G) >= tile_u0 ? 0 : 1);
               uint64_t* src = p.ws + slot * BN * kBM + row;
-              uint64_t v[(BN + 31) / 32][kCols];
-              const uint64_t t0 = globaltimer_ns();
-              while (true) {
+              // one round polls every word of a 32-column chunk at once
 #pragma unroll
-                for (int cb = 0; cb < (BN + 31) / 32; ++cb)
+              for (int cb = 0; cb < (BN + 31) / 32; ++cb) {
+                uint64_t v[kCols];
+                const uint64_t t0 = globaltimer_ns();
+                while (true) {
 #pragma unroll
                   for (int i = 0; i < kCols; ++i) {
                     const int mm = cb * 32 + i;
-                    v[cb][i] = q0 + mm < M ? ld_word(src + (int64_t)mm * kBM) : (uint64_t)kFullTag << 32;
+                    v[i] = q0 + mm < M ? ld_word(src + (int64_t)mm * kBM) : (uint64_t)kFullTag << 32;
                   }
-                uint32_t all = 1;
+                  uint32_t all = 1;
 #pragma unroll
-                for (int cb = 0; cb < (BN + 31) / 32; ++cb)
-#pragma unroll
-                  for (int i = 0; i < kCols; ++i) all &= (uint32_t)((v[cb][i] >> 32) == kFullTag);
-                if (all) break;
-                if (globaltimer_ns() - t0 > p.timeout_ns) {
-                  atomicCAS(p.err, 0u, kErrTimeout);
-                  ok_all = false;
-                  break;
+                  for (int i = 0; i < kCols; ++i) all &= (uint32_t)((v[i] >> 32) == kFullTag);
+                  if (all) break;
+                  if (globaltimer_ns() - t0 > p.timeout_ns) {
+                    atomicCAS(p.err, 0u, kErrTimeout);
+                    ok_all = false;
+                    break;
+                  }
                 }
-              }
-#pragma unroll
-              for (int cb = 0; cb < (BN + 31) / 32; ++cb)
+                if (!ok_all) break;
 #pragma unroll
                 for (int i = 0; i < kCols; ++i) {
                   const int mm = cb * 32 + i;
-                  sum[cb][i] = __fadd_rn(sum[cb][i], __uint_as_float((uint32_t)v[cb][i]));
+                  sum[cb][i] = __fadd_rn(sum[cb][i], __uint_as_float((uint32_t)v[i]));
                   if (q0 + mm < M) st_word(src + (int64_t)mm * kBM, 0ull);     // empty again
                 }
+              }
             }
             if (n < N && ok_all) {
 #pragma unroll
@@ -785,7 +738,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
       first_item = false;
     }
     if (tma_store && et == 0) bulk_wait_group<0>();   // stores done before the CTA's smem goes away
-  } else if (C::kSplitCopy) {
+  } else {
     // ------------------------------------------------------------ scale copies
     // warp 6 copies P's scale chunks of each stage into TMEM, warp 7 + rb the
     // chunks of Q's 128-row block rb; each then commits to the stage's
@@ -816,12 +769,13 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
             tc_fence_after();
           }
           const uint32_t sfa_t = sf_t0 + region * C::kSfStageCols;
-          const int nkb = min(4, kc - 4 * k);
+          const int nkb = min(C::kKB, kc - C::kKB * k);
           if (copy_p) {
             const uint64_t d = desc0 + (uint64_t)((stage * C::kSfaBytes) >> 4);
-            if (nkb == 4) {
+            if (nkb == C::kKB) {
 #pragma unroll
-              for (int kb = 0; kb < 4; ++kb) tc_cp_32x128b_warpx4(sfa_t + kb * 4, d + (uint64_t)(kb * (kSfChunk >> 4)));
+              for (int kb = 0; kb < C::kKB; ++kb)
+                tc_cp_32x128b_warpx4(sfa_t + kb * 4, d + (uint64_t)(kb * (kSfChunk >> 4)));
             } else {
               for (int kb = 0; kb < nkb; ++kb) tc_cp_32x128b_warpx4(sfa_t + kb * 4, d + (uint64_t)(kb * (kSfChunk >> 4)));
             }
@@ -830,7 +784,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
             const uint32_t sfb_t = sfa_t + C::kSfaCols;
             for (int kb = 0; kb < nkb; ++kb)
               tc_cp_32x128b_warpx4(sfb_t + kb * 4 * C::kSfbBlocks + rbq * 4,
-                                   d + (uint64_t)((rbq * 4 + kb) * (kSfChunk >> 4)));
+                                   d + (uint64_t)((rbq * C::kKB + kb) * (kSfChunk >> 4)));
           }
           tc_commit(bar_sf + 8 * stage);
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
@@ -879,17 +833,18 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Codes of a [rows, K/2]-byte operand, 128-byte x box_rows boxes, 128B swizzle.
-bool make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int box_rows) {
+// Codes of a [rows, K/2]-byte operand in boxes of row_bytes x box_rows, with
+// the matching swizzle (128-byte rows: 128B, 64-byte rows: 64B).
+bool make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int box_rows, int row_bytes) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-  const cuuint32_t box[2] = {(cuuint32_t)kBKBytes, (cuuint32_t)box_rows};
+  const cuuint32_t box[2] = {(cuuint32_t)row_bytes, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            CU_TENSOR_MAP_INTERLEAVE_NONE, row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Output [M, N] (bf16 or f32), boxes of 128 rows x 128 bytes, 128B swizzle.
@@ -1011,7 +966,9 @@ nvfp4_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float ga,
   const uint8_t* codes_q = swap ? a_codes : w_codes;
   p.sf_p = swap ? w_scales : a_scales;
   p.sf_q = swap ? a_scales : w_scales;
-  if (!make_code_map(&p.tmap_p, codes_p, p.rows_p, K, kBM) || !make_code_map(&p.tmap_q, codes_q, p.rows_q, K, bn))
+  const int kkb = swap ? Cfg<16, true>::kKB : Cfg<256, false>::kKB;
+  if (!make_code_map(&p.tmap_p, codes_p, p.rows_p, K, kBM, 32 * kkb) ||
+      !make_code_map(&p.tmap_q, codes_q, p.rows_q, K, bn, 32 * kkb))
     return NVFP4_ERR_CUDA;
   p.out = out;
   // TMA stores need 16-byte aligned output rows
@@ -1024,7 +981,7 @@ nvfp4_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float ga,
   p.N = N;
   p.rb_q = (int)ceil_div(p.rows_q, 128);
   p.kc = (int)ceil_div(K, 64);
-  p.kt = (int)ceil_div(K, 256);
+  p.kt = (int)ceil_div(K, 64 * kkb);
   p.tiles_p = (int)ceil_div(p.rows_p, kBM);
   p.tiles_q = (int)ceil_div(p.rows_q, bn);
   p.n_seg = n_seg;
@@ -1124,7 +1081,9 @@ nvfp4_status run_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_scales, f
   p.rows_q = (int)M;
   p.sf_p = w_scales;
   p.sf_q = a_scales;
-  if (!make_code_map(&p.tmap_p, w_codes, p.rows_p, K, kBM) || !make_code_map(&p.tmap_q, a_codes, p.rows_q, K, bn))
+  constexpr int kkb = Cfg<16, true>::kKB;
+  if (!make_code_map(&p.tmap_p, w_codes, p.rows_p, K, kBM, 32 * kkb) ||
+      !make_code_map(&p.tmap_q, a_codes, p.rows_q, K, bn, 32 * kkb))
     return NVFP4_ERR_CUDA;
   p.out = out;
   p.tma_store = 0;
@@ -1134,7 +1093,7 @@ nvfp4_status run_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_scales, f
   p.N = N;
   p.rb_q = (int)ceil_div(p.rows_q, 128);
   p.kc = (int)ceil_div(K, 64);
-  p.kt = (int)ceil_div(K, 256);
+  p.kt = (int)ceil_div(K, 64 * kkb);
   p.tiles_p = (int)ceil_div(p.rows_p, kBM);
   p.tiles_q = 1;
   p.n_seg = 1;
