@@ -113,8 +113,8 @@ struct Cfg {
   static constexpr int kOffMisc = kOffSeg + 2 * 4 * NVFP4_MAX_SEGMENTS;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;            // + alignment slack
   // TMEM columns.  Normal 128x256 tiles: the copy warps run ahead of the
-  // MMAs, so the scales of successive steps use a ring of two regions at the
-  // top of TMEM ([416,512) for 48-column regions); the two accumulator
+  // MMAs, so the scales of successive steps use a ring of regions at the top
+  // of TMEM ([320,512) for four 48-column regions); the two accumulator
   // buffers, [0,256) and [kAcc1Col, kAcc1Col + 256), fill the rest and
   // overlap, so tile t+1 can start as soon as the epilogue has drained the
   // shared columns of tile t (it drains those 64-column slots first).
@@ -125,7 +125,9 @@ struct Cfg {
   static constexpr int kSfaCols = 4 * kKB;                           // kKB MMAs x 4 columns
   static constexpr int kSfbCols = kSfbBlocks * 4 * kKB;
   static constexpr int kSfStageCols = kSfaCols + kSfbCols;
-  static constexpr int kSfRegions = kOverlapAcc ? 2 : kStages;
+  // four regions (192 columns) let the copy warps run up to three steps
+  // ahead; the accumulators then share 192 columns (3 slots drained first)
+  static constexpr int kSfRegions = kOverlapAcc ? 4 : kStages;
   static constexpr int kSfBase = kOverlapAcc ? kTmemCols - kSfRegions * kSfStageCols : kAccCols;
   static constexpr int kAcc1Col = kOverlapAcc ? kSfBase - 256 : 0;
   static constexpr int kSharedSlots = kOverlapAcc ? (256 - kAcc1Col + 63) / 64 : 0;   // drained before release
