@@ -173,6 +173,9 @@ class Decode:
         self.gemm_bytes = M * K // 2 + M * K // 16 + N * K // 2 + N * K // 16 + M * N * 2
         self.quant_bytes = M * K * 2 + M * K // 2 + M * K // 16
         self.step_bytes = self.gemm_bytes + self.quant_bytes
+        # the whole layer in one kernel: X in, W in, output out (the
+        # quantized activation never leaves the chip)
+        self.layer_bytes = M * K * 2 + N * K // 2 + N * K // 16 + M * N * 2
         self.launches_per_step = 2
 
     def step(self, i):
@@ -186,6 +189,19 @@ class Decode:
         w = self.w
         wc, ws = self.w_copies[i % self.n_copies]
         self.nv.nvfp4_gemm(self.a_codes, self.a_sc, self.ga, wc, ws, self.gw, w.M, w.N, w.K, self.out)
+
+    def linear(self, i):
+        # the layer through its public call: quantize X into the activation
+        # buffers, block-scaled GEMM, dequantizing epilogue (two kernels)
+        w = self.w
+        wc, ws = self.w_copies[i % self.n_copies]
+        self.nv.nvfp4_linear(self.x, self.ga, wc, ws, self.gw, w.N, self.out, self.a_codes, self.a_sc)
+
+    def linear_one_kernel(self, i):
+        # the same layer as one kernel that quantizes X in shared memory
+        w = self.w
+        wc, ws = self.w_copies[i % self.n_copies]
+        self.nv.nvfp4_linear(self.x, self.ga, wc, ws, self.gw, w.N, self.out)
 
     def config(self):
         w = self.w
@@ -392,25 +408,31 @@ def run_reference(args):
 
 def measure_decode(torch, nv, synth, dev, rank, world, l2, args, stream, barrier, max_over_ranks, peaks,
                    peak_kind):
+    """Headline: the decode-shape linear layer as one step = nvfp4_linear
+    (quantize X, block-scaled GEMM, dequantizing epilogue: the quantize
+    kernel then the GEMM).  Also timed: the same call in its one-kernel form
+    and the GEMM alone."""
     d = Decode(torch, nv, synth, dev, rank, l2)
     torch.cuda.synchronize()
     # soak so the clock sampler sees the GPU under this load before timing
     t_soak = time.time()
     i = 0
     while time.time() - t_soak < args.soak:
-        d.step(i)
+        d.linear(i)
         i += 1
         if i % 64 == 0:
             torch.cuda.synchronize()
     barrier()
     with torch.cuda.stream(stream):
-        ms_step, g_step = time_graph(torch, d.step, args.steps, args.warmup, stream)
+        ms_lin, g_lin = time_graph(torch, d.linear, args.steps, args.warmup, stream)
+        ms_one, g_one = time_graph(torch, d.linear_one_kernel, args.steps, args.warmup, stream)
         ms_gemm, g_gemm = time_graph(torch, d.gemm_only, args.steps, args.warmup, stream)
     barrier()
     t_end = time.time()
-    ms_step = max_over_ranks(ms_step)
+    ms_lin = max_over_ranks(ms_lin)
+    ms_one = max_over_ranks(ms_one)
     ms_gemm = max_over_ranks(ms_gemm)
-    del g_step, g_gemm
+    del g_lin, g_one, g_gemm
 
     # end to end through the public API: pinned host X in, host result out
     x_host = d.x.cpu().pin_memory()
@@ -420,23 +442,23 @@ def measure_decode(torch, nv, synth, dev, rank, world, l2, args, stream, barrier
     def e2e_step(i):
         x_dev.copy_(x_host, non_blocking=True)
         wc, ws = d.w_copies[i % d.n_copies]
-        nv.nvfp4_quantize(x_dev, d.ga, d.a_codes, d.a_sc)
-        nv.nvfp4_gemm(d.a_codes, d.a_sc, d.ga, wc, ws, d.gw, d.w.M, d.w.N, d.w.K, d.out)
+        nv.nvfp4_linear(x_dev, d.ga, wc, ws, d.gw, d.w.N, d.out, d.a_codes, d.a_sc)
         out_host.copy_(d.out, non_blocking=True)
 
     barrier()
     ms_e2e = max_over_ranks(time_eager(torch, e2e_step, args.steps, args.warmup))
     barrier()
 
-    value = aggregate_replicas(ms_step, d.step_bytes, world)[1] / 1e9
+    value = aggregate_replicas(ms_lin, d.step_bytes, world)[1] / 1e9
     gemm_gbs = d.gemm_bytes / (ms_gemm * 1e-3) / 1e9
     hbm_peak = float(peaks["hbm_gbs"])
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_lin, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, e4m3 block scales, f32 accumulate, bf16 out)",
         "data": "synthetic (seeded; decode X N(0,1) with 0.1% channels x60, W N(0,0.02))",
-        "config": dict(d.config(), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+        "config": dict(d.config(), step="nvfp4_linear: quantize kernel + GEMM kernel (with epilogue)",
+                       parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
         "roofline": {"bound": "hbm", "kernel": "nvfp4_gemm_kernel<16,swap>", "achieved": gemm_gbs,
                      "peak": hbm_peak, "unit": "GB/s", "frac": gemm_gbs / hbm_peak,
                      "peak_kind": f"{peak_kind} copy bandwidth",
@@ -446,6 +468,10 @@ def measure_decode(torch, nv, synth, dev, rank, world, l2, args, stream, barrier
                 "ms_per_step": ms_e2e, "h2d_bytes_per_step": d.x.numel() * d.x.element_size(),
                 "d2h_bytes_per_step": d.out.numel() * d.out.element_size()},
         "gpu_launches": d.launches_per_step * args.steps,
+        "decode_one_kernel": {
+            "step": "nvfp4_linear without activation buffers: one kernel quantizes X in shared memory",
+            "ms_per_step": ms_one, "GB/s": world * d.layer_bytes / (ms_one * 1e-3) / 1e9,
+            "bytes_per_step": d.layer_bytes},
     }
     del d
     return line, t_soak, t_end

@@ -155,6 +155,29 @@ NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scale
                         int64_t M, int64_t N, int64_t K, void* out, nvfp4_out_dtype out_dtype,
                         nvfp4_stream_t stream);
 
+/* The whole W4A4 linear layer: quantize the activation with a_global_scale
+ * (as nvfp4_quantize, TCGEN05 scales) and multiply by the quantized weight
+ * (as nvfp4_gemm) [picx.dev summary, "Background": activations and weights
+ * both in NVFP4, native 4-bit tensor-core GEMM].
+ *   x       device [M, K] row-major, bf16 or f32 per x_dtype
+ *   w_*     as nvfp4_gemm; N output features; out as nvfp4_gemm
+ *   a_codes, a_scales: device buffers for the quantized activation
+ *           ([M, K/2] bytes and nvfp4_scale_bytes(M, K, NVFP4_SF_TCGEN05)),
+ *           or both NULL.
+ * With the buffers the call is exactly nvfp4_quantize into them followed by
+ * nvfp4_gemm.  Without them, for M <= 32 when every CTA's share of the
+ * K-split work fits in 16 K-steps of 256 (decode shapes), one kernel
+ * quantizes x into shared memory itself and runs the GEMM, writing no
+ * activation to memory; its result is bitwise equal to the two-call form
+ * (same arithmetic, same K split, same summation order).  Workspace and
+ * capture rules as nvfp4_gemm.
+ * Errors: INVALID_ARG (also: NULL buffers for a shape the one-kernel form
+ * does not cover), ALIGNMENT, UNSUPPORTED, CUDA. */
+NVFP4_API nvfp4_status nvfp4_linear(const void* x, nvfp4_in_dtype x_dtype, int64_t M, int64_t K,
+                          float a_global_scale, const uint8_t* w_codes, const uint8_t* w_scales,
+                          float w_global_scale, int64_t N, void* out, nvfp4_out_dtype out_dtype,
+                          uint8_t* a_codes, uint8_t* a_scales, nvfp4_stream_t stream);
+
 /* nvfp4_gemm for decode-sized M that allocates nothing.  The pages have no
  * counterpart: this is an interface variant, not part of the method.  It
  * computes exactly what nvfp4_gemm computes for the same arguments (same

@@ -45,6 +45,8 @@ _lib.nvfp4_amax.argtypes = [_vp, ctypes.c_int, _i64, _i64, _vp, _vp]
 _lib.nvfp4_quantize.argtypes = [_vp, ctypes.c_int, _i64, _i64, _f32, _vp, _vp, ctypes.c_int, _vp, _vp]
 _lib.nvfp4_swizzle_scales.argtypes = [_vp, _i64, _i64, _vp, _vp]
 _lib.nvfp4_gemm.argtypes = [_vp, _vp, _f32, _vp, _vp, _f32, _i64, _i64, _i64, _vp, ctypes.c_int, _vp]
+_lib.nvfp4_linear.argtypes = [_vp, ctypes.c_int, _i64, _i64, _f32, _vp, _vp, _f32, _i64, _vp, ctypes.c_int, _vp, _vp,
+                              _vp]
 _lib.nvfp4_gemm_noalloc.argtypes = [_vp, _vp, _f32, _vp, _vp, _f32, _i64, _i64, _i64, _vp, ctypes.c_int, _vp]
 _lib.nvfp4_fused_proj.argtypes = [_vp, _vp, _f32, _vp, _vp, ctypes.POINTER(_i64), ctypes.POINTER(_f32),
                                   ctypes.c_int, _i64, _i64, _vp, ctypes.c_int, _vp]
@@ -147,6 +149,16 @@ def nvfp4_gemm(a_codes, a_scales, a_global_scale, w_codes, w_scales, w_global_sc
     _check("nvfp4_gemm", _lib.nvfp4_gemm(_ptr(a_codes), _ptr(a_scales), float(a_global_scale), _ptr(w_codes),
                                          _ptr(w_scales), float(w_global_scale), M, N, K, _ptr(out),
                                          _out_dtype(out), _stream(out)))
+
+
+def nvfp4_linear(x: torch.Tensor, a_global_scale, w_codes, w_scales, w_global_scale, N, out: torch.Tensor,
+                 a_codes=None, a_scales=None) -> None:
+    M, K = x.shape
+    _check("nvfp4_linear",
+           _lib.nvfp4_linear(_ptr(x), _in_dtype(x), M, K, float(a_global_scale), _ptr(w_codes), _ptr(w_scales),
+                             float(w_global_scale), N, _ptr(out), _out_dtype(out),
+                             _ptr(a_codes) if a_codes is not None else None,
+                             _ptr(a_scales) if a_scales is not None else None, _stream(out)))
 
 
 def nvfp4_gemm_noalloc(a_codes, a_scales, a_global_scale, w_codes, w_scales, w_global_scale, M, N, K,

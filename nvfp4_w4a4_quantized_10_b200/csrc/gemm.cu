@@ -39,6 +39,7 @@
 #include <mutex>
 #include <utility>
 
+#include "block_quant.cuh"
 #include "common.h"
 #include "ptx.cuh"
 
@@ -71,10 +72,20 @@ struct alignas(64) GemmParams {
   int n_seg;
   int seg_end[NVFP4_MAX_SEGMENTS];
   float seg_alpha[NVFP4_MAX_SEGMENTS];
+  // activation quantized in the kernel (swapped tiles only): X [M, K]
+  // row-major, its global scale, K
+  const void* x;
+  float x_gs;
+  int64_t K;
 };
 
-template <int BN, bool SWAP>
+// QX: 0 = the Q operand (activations) arrives quantized, as codes and scales
+// in global memory; 1 / 2 = swapped tiles whose activation X (bf16 / f32) the
+// kernel quantizes itself into shared memory, all of the CTA's K-steps at
+// once, before the first MMA.
+template <int BN, bool SWAP, int QX = 0>
 struct Cfg {
+  static constexpr bool kQx = QX != 0;
   // K per pipeline step: kKB blocks of 64 (one MMA each), 256 deep, as
   // 128-byte rows with the 128B swizzle.  (128-deep steps with 64-byte rows
   // and the 64B swizzle also work, and fit twice as many stages, but measured
@@ -86,19 +97,27 @@ struct Cfg {
   static constexpr uint32_t kSbo = 8 * kRowBytes;                    // bytes between 8-row groups
   static constexpr int kSfbBlocks = (BN + 127) / 128;                // 128-row scale blocks of Q
   static constexpr int kABytes = kBM * kRowBytes;
-  static constexpr int kBBytes = BN * kRowBytes;
+  static constexpr int kBBytes = kQx ? 0 : BN * kRowBytes;           // Q codes per stage
   static constexpr int kSfaBytes = kKB * kSfChunk;
-  static constexpr int kSfbBytes = kSfbBlocks * kKB * kSfChunk;
+  static constexpr int kSfbBytes = kQx ? 0 : kSfbBlocks * kKB * kSfChunk;
   static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
   static constexpr int kOutBytes = SWAP ? 0 : 2 * kStageOutBytes;    // double-buffered output sub-tiles
+  // in-kernel activation: codes (BN rows x 128 B, 128B swizzle) and one
+  // 128-row scale block per K-step, for up to kActSteps steps
+  static constexpr int kActSteps = kQx ? 16 : 0;
+  static constexpr int kActCodeBytes = BN * kRowBytes;
+  static constexpr int kActSfBytes = kKB * kSfChunk;
+  static constexpr int kActBytes = kActSteps * (kActCodeBytes + kActSfBytes);
   static constexpr int kMaxStages = 8;
-  static constexpr int kFit = (222 * 1024 - kOutBytes) / kStageBytes;
+  static constexpr int kFit = (222 * 1024 - kOutBytes - kActBytes) / kStageBytes;
   static constexpr int kStages = kFit < kMaxStages ? kFit : kMaxStages;
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + kStages * kABytes;
   static constexpr int kOffSfa = kOffB + kStages * kBBytes;
   static constexpr int kOffSfb = kOffSfa + kStages * kSfaBytes;
-  static constexpr int kOffOut = kOffSfb + kStages * kSfbBytes;      // 1024-aligned
+  static constexpr int kOffAct = kOffSfb + kStages * kSfbBytes;      // 1024-aligned
+  static constexpr int kOffActSf = kOffAct + kActSteps * kActCodeBytes;
+  static constexpr int kOffOut = kOffActSf + kActSteps * kActSfBytes;   // 1024-aligned
   static constexpr int kOffBar = kOffOut + kOutBytes;
   // Extra warps issue the scale copies (warp 6: P's scales, warp 7 + rb: the
   // scales of Q's 128-row block rb) so that the MMA warp issues only MMAs; a
@@ -107,11 +126,13 @@ struct Cfg {
   static constexpr int kCopyWarps = 1 + kSfbBlocks;
   static constexpr int kThreads = 192 + 32 * kCopyWarps;
   // full, empty, acc_full, acc_empty, drain, one scales-ready barrier per
-  // stage and one drain barrier per copy warp
-  static constexpr int kNumBars = 2 * kStages + 3 + kStages + kCopyWarps;
+  // stage, one drain barrier per copy warp, and (in-kernel activation) one
+  // activation-ready barrier per K-step
+  static constexpr int kNumBars = 2 * kStages + 3 + kStages + kCopyWarps + kActSteps;
   static constexpr int kOffSeg = kOffBar + kNumBars * 8;             // segment table: ends, alphas
   static constexpr int kOffMisc = kOffSeg + 2 * 4 * NVFP4_MAX_SEGMENTS;
-  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;            // + alignment slack
+  static constexpr int kOffRtab = kOffMisc + 16;                     // in-kernel activation: g / e4m3(s)
+  static constexpr int kSmemBytes = kOffRtab + (kQx ? 1024 : 0) + 1024;   // + alignment slack
   // TMEM columns.  Normal 128x256 tiles: the copy warps run ahead of the
   // MMAs, so the scales of successive steps use a ring of regions at the top
   // of TMEM ([320,512) for four 48-column regions); the two accumulator
@@ -136,6 +157,8 @@ struct Cfg {
   static_assert(kSfBase + kSfRegions * kSfStageCols <= kTmemCols, "TMEM budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(BN % 16 == 0 && BN <= 256, "MMA N");
+  static_assert(!kQx || (SWAP && BN <= 32), "in-kernel activation: swapped tiles, M <= 32");
+  static_assert(kOffAct % 1024 == 0 && kActCodeBytes % 1024 == 0, "activation tiles on swizzle atoms");
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -242,9 +265,10 @@ __device__ __forceinline__ uint64_t ld_word(const uint64_t* p) {
 // stored with the 128B swizzle the output tensor map uses.
 __device__ __forceinline__ uint32_t swz128(uint32_t r, uint32_t c) { return r * 128 + ((c ^ (r & 7)) << 4); }
 
-template <int BN, bool SWAP, bool OUT_F32>
-__global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(const __grid_constant__ GemmParams p) {
-  using C = Cfg<BN, SWAP>;
+template <int BN, bool SWAP, bool OUT_F32, int QX = 0>
+__global__ void __launch_bounds__(Cfg<BN, SWAP, QX>::kThreads, 1)
+    nvfp4_gemm_kernel(const __grid_constant__ GemmParams p) {
+  using C = Cfg<BN, SWAP, QX>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -255,6 +279,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
   const uint32_t bar_drain = bar_acc_empty + 8;
   const uint32_t bar_sf = bar_drain + 8;                     // [kStages]
   const uint32_t bar_cp_drain = bar_sf + 8 * C::kStages;     // [kCopyWarps]
+  const uint32_t bar_act = bar_cp_drain + 8 * C::kCopyWarps;  // [kActSteps] in-kernel activation ready
   int* seg_end_s = reinterpret_cast<int*>(smem + C::kOffSeg);
   float* seg_alpha_s = reinterpret_cast<float*>(smem + C::kOffSeg + 4 * NVFP4_MAX_SEGMENTS);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
@@ -276,6 +301,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
     mbar_init(bar_drain, 1);
     for (int s = 0; s < C::kStages; ++s) mbar_init(bar_sf + 8 * s, C::kCopyWarps);
     for (int i = 0; i < C::kCopyWarps; ++i) mbar_init(bar_cp_drain + 8 * i, 1);
+    for (int j = 0; j < C::kActSteps; ++j) mbar_init(bar_act + 8 * j, 128);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&p.tmap_p);
@@ -340,7 +366,8 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
       };
       auto expect = [&](int stage, int q0, int k) {
         const uint32_t sf_bytes = (uint32_t)min(C::kKB, kc - C::kKB * k) * kSfChunk;
-        mbar_arrive_expect_tx(bar_full + 8 * stage, C::kABytes + C::kBBytes + sf_bytes * (1 + nsfb_of(q0)));
+        mbar_arrive_expect_tx(bar_full + 8 * stage,
+                              C::kABytes + C::kBBytes + sf_bytes * (1 + (C::kQx ? 0 : nsfb_of(q0))));
       };
       const WorkIter w0 = work_begin(p, SWAP);
       // prologue: the first kStages stages are free
@@ -359,7 +386,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
       for_steps(w0, 0, npro, [&](int j, int p0, int q0, int k) {
         expect(j, q0, k);
         load_p(j, p0, k);
-        load_q(j, q0, k);
+        if (!C::kQx) load_q(j, q0, k);
         issued_mask |= 1u << j;
       });
       int stage = npro % C::kStages;
@@ -370,7 +397,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, p.err, p.timeout_ns)) { ok = false; return; }
           expect(stage, q0, k);
           load_p(stage, p0, k);
-          load_q(stage, q0, k);
+          if (!C::kQx) load_q(stage, q0, k);
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         });
@@ -392,10 +419,10 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
     // Descriptors of stage 0, k-block 0; later stages and k-blocks only move
     // the 14-bit start-address field (address >> 4), which never carries.
     const uint64_t a_desc0 = smem_desc(sbase + C::kOffA, 16, C::kSbo, C::kSwizzleLayout);
-    const uint64_t b_desc0 = smem_desc(sbase + C::kOffB, 16, C::kSbo, C::kSwizzleLayout);
+    const uint64_t b_desc0 = smem_desc(sbase + (C::kQx ? C::kOffAct : C::kOffB), 16, C::kSbo, C::kSwizzleLayout);
     const uint32_t sf_t0 = tmem_base + C::kSfBase;
     const int kc = p.kc;
-    int stage = 0, region = 0;
+    int stage = 0, region = 0, lstep = 0;    // lstep: steps of this CTA so far
     uint32_t phase = 0, acc_phase = 0, acc_buf = 0;
     bool ok = true;
     WorkIter w = work_begin(p, SWAP);
@@ -405,13 +432,19 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
       tc_fence_after();
       const uint32_t acc = tmem_base + (acc_buf ? C::kAcc1Col : 0);
       for (int k = kb0; k < ke0; ++k) {
+        if (C::kQx && lstep >= C::kActSteps) {     // the host sizes the grid so this cannot happen
+          atomicCAS(p.err, 0u, kErrBounds);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
         if (!mbar_wait(bar_sf + 8 * stage, phase, abort_flag, p.err, p.timeout_ns)) { ok = false; break; }
         tc_fence_after();
         if (lane == 0) {
           const uint32_t sfa_t = sf_t0 + region * C::kSfStageCols;
           const uint32_t sfb_t = sfa_t + C::kSfaCols;
           const uint64_t ad = a_desc0 + (uint64_t)((stage * C::kABytes) >> 4);
-          const uint64_t bd = b_desc0 + (uint64_t)((stage * C::kBBytes) >> 4);
+          const uint64_t bd = b_desc0 + (uint64_t)(((C::kQx ? lstep * C::kActCodeBytes : stage * C::kBBytes)) >> 4);
           const uint32_t acc_in = k != kb0 ? 1u : 0u;
           const int nkb = min(C::kKB, kc - C::kKB * k);
           if (nkb == C::kKB) {
@@ -429,6 +462,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
         __syncwarp();
         if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         if (++region == C::kSfRegions) region = 0;
+        ++lstep;
       }
       if (!ok) break;
       if (lane == 0) tc_commit(bar_acc_full);
@@ -459,6 +493,89 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
     const int64_t U = (int64_t)p.tiles_p * p.kt, G = gridDim.x;
     int tp, tq, kb0, ke0;
     bool first_item = true;
+    if constexpr (C::kQx) {
+      // ---------------------------------------------- in-kernel activation
+      // Quantize the rows of X for every K-step this CTA computes, with the
+      // same per-block arithmetic as the quantize kernel, into the MMA's
+      // operand layout: codes of step j at kOffAct + j * BN * 128 (row m at
+      // m * 128, 16-byte chunks 128B-swizzled), scales of step j at
+      // kOffActSf + j * 2048 (the 512-byte chunk of K-block kb holds row m's
+      // four scales at m * 16).  Rows [M, BN) and K past the end stay zero.
+      constexpr bool kF32 = QX == 2;
+      constexpr int kEsz = kF32 ? 4 : 2;
+      // the K-steps of this CTA, in the order every role walks them
+      int ks[C::kActSteps];
+      int nsteps = 0;
+      {
+        WorkIter wq = work_begin(p, SWAP);
+        int a, b2, c0, c1;
+        while (work_next(p, wq, a, b2, c0, c1))
+          for (int k = c0; k < c1 && nsteps < C::kActSteps; ++k) ks[nsteps++] = k;
+      }
+      const int64_t K = p.K;
+      const uint8_t* xb = reinterpret_cast<const uint8_t*>(p.x);
+      // A thread owns (row, block) pairs et, et + 128, ... (one pair when
+      // M <= 8) and handles them one after the other.  Per pair, windows of
+      // kWin steps: the next window's loads are in flight while the current
+      // one is quantized (all its blocks together, for instruction-level
+      // parallelism: four warps alone cannot hide latency by switching).  A
+      // thread publishes step j (its barrier, 128 arrivals) after its last
+      // pair's block of step j is stored, so the MMAs can start early.
+      constexpr int kWin = kF32 ? 2 : 4;
+      const int npairs = (int)M * 16;
+      const int nq = et < npairs ? (npairs - 1 - et) / 128 + 1 : 0;   // pairs of this thread
+      asm volatile("griddepcontrol.wait;" ::: "memory");      // X is written by the previous kernel
+      auto load_window = [&](int pair, int j0, Block16<kF32> (&B)[kWin]) {
+        const int m = pair >> 4, bq = pair & 15;
+#pragma unroll
+        for (int u = 0; u < kWin; ++u) {
+          const int jj = j0 + u;
+          const int64_t e = (int64_t)(jj < nsteps ? ks[jj] : 0) * 256 + bq * 16;
+          if (jj < nsteps && e < K) load_block_at<kF32>(xb + ((int64_t)m * K + e) * kEsz, B[u]);
+        }
+      };
+      Block16<kF32> Bc[kWin], Bn[kWin];
+      if (nq > 0) load_window(et, 0, Bc);
+      float* rtab = reinterpret_cast<float*>(smem + C::kOffRtab);
+      rtab[et] = recip_entry(p.x_gs, (uint32_t)et);
+      rtab[et + 128] = recip_entry(p.x_gs, (uint32_t)et + 128);
+      for (int i = et; i < C::kActBytes / 16; i += 128)
+        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(sbase + C::kOffAct + 16 * i), "r"(0) : "memory");
+      named_bar_sync(kEpiBar, 128);                // zeros and rtab are in place
+      if (nq == 0)
+        for (int jj = 0; jj < nsteps; ++jj) mbar_arrive(bar_act + 8 * jj);
+      for (int q = 0; q < nq; ++q) {
+        const int pair = et + 128 * q;
+        const int m = pair >> 4, bq = pair & 15;
+        const bool last = q == nq - 1;
+        for (int j0 = 0; j0 < nsteps; j0 += kWin) {
+          // prefetch: the next window of this pair, or the first of the next pair
+          if (j0 + kWin < nsteps) load_window(pair, j0 + kWin, Bn);
+          else if (!last) load_window(pair + 128, 0, Bn);
+#pragma unroll
+          for (int u = 0; u < kWin; ++u) {
+            const int jj = j0 + u;
+            const int64_t e = (int64_t)(jj < nsteps ? ks[jj] : 0) * 256 + bq * 16;
+            if (jj < nsteps && e < K) {
+              uint32_t lo, hi;
+              const uint32_t sc = quantize_block<kF32>(Bc[u], p.x_gs, rtab, lo, hi);
+              // byte bq * 8 of row m: 16-byte chunk bq / 2, swizzled with m % 8
+              *reinterpret_cast<uint2*>(smem + C::kOffAct + jj * C::kActCodeBytes + m * 128 +
+                                        ((((bq >> 1) ^ (m & 7))) << 4) + (bq & 1) * 8) = make_uint2(lo, hi);
+              smem[C::kOffActSf + jj * C::kActSfBytes + (bq >> 2) * kSfChunk + m * 16 + (bq & 3)] = (uint8_t)sc;
+            }
+          }
+          if (last) {
+            fence_proxy_async_smem();              // generic-proxy writes -> tcgen05 reads
+#pragma unroll
+            for (int u = 0; u < kWin; ++u)
+              if (j0 + u < nsteps) mbar_arrive(bar_act + 8 * (j0 + u));
+          }
+#pragma unroll
+          for (int u = 0; u < kWin; ++u) Bc[u] = Bn[u];
+        }
+      }
+    }
     while (work_next(p, w, tp, tq, kb0, ke0)) {
       const int64_t p0 = (int64_t)tp * kBM, q0 = (int64_t)tq * BN;
       if (!mbar_wait(bar_acc_full, acc_phase, abort_flag, p.err, p.timeout_ns)) break;
@@ -749,7 +866,8 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
     const bool copy_p = warp == 6;
     const int rbq = warp - 7;                   // Q block of this warp
     if (lane == 0) {
-      const uint64_t desc0 = smem_desc(sbase + (copy_p ? C::kOffSfa : C::kOffSfb), 16, 128, 0);
+      const uint64_t desc0 =
+          smem_desc(sbase + (copy_p ? C::kOffSfa : (C::kQx ? C::kOffActSf : C::kOffSfb)), 16, 128, 0);
       const uint32_t sf_t0 = tmem_base + C::kSfBase;
       const int kc = p.kc;
       int stage = 0, region = 0;
@@ -760,6 +878,12 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
       int tp, tq, kb0, ke0;
       while (ok && work_next(p, w, tp, tq, kb0, ke0)) {
         for (int k = kb0; k < ke0; ++k) {
+          if (C::kQx && step >= C::kActSteps) { ok = false; break; }
+          // in-kernel activation: this step's scales are written by the epilogue warps
+          if (C::kQx && !copy_p && !mbar_wait(bar_act + 8 * (int)step, 0, abort_flag, p.err, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
           if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, p.err, p.timeout_ns)) { ok = false; break; }
           if (C::kSfRegions < C::kStages && step >= C::kSfRegions) {
             // the MMAs of step - kSfRegions read this region: wait for their
@@ -782,7 +906,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP>::kThreads, 1) nvfp4_gemm_kernel(
               for (int kb = 0; kb < nkb; ++kb) tc_cp_32x128b_warpx4(sfa_t + kb * 4, d + (uint64_t)(kb * (kSfChunk >> 4)));
             }
           } else {
-            const uint64_t d = desc0 + (uint64_t)((stage * C::kSfbBytes) >> 4);
+            const uint64_t d = desc0 + (uint64_t)((C::kQx ? step * C::kActSfBytes : stage * C::kSfbBytes) >> 4);
             const uint32_t sfb_t = sfa_t + C::kSfaCols;
             for (int kb = 0; kb < nkb; ++kb)
               tc_cp_32x128b_warpx4(sfb_t + kb * 4 * C::kSfbBlocks + rbq * 4,
@@ -895,10 +1019,10 @@ cudaError_t get_workspace(const DeviceInfo* d, cudaStream_t st, Workspace* out) 
   return cudaSuccess;
 }
 
-template <int BN, bool SWAP, bool OUT_F32>
+template <int BN, bool SWAP, bool OUT_F32, int QX = 0>
 cudaError_t launch(const GemmParams& p, const DeviceInfo* d, cudaStream_t st) {
-  using Cf = Cfg<BN, SWAP>;
-  auto kern = nvfp4_gemm_kernel<BN, SWAP, OUT_F32>;
+  using Cf = Cfg<BN, SWAP, QX>;
+  auto kern = nvfp4_gemm_kernel<BN, SWAP, OUT_F32, QX>;
   static std::once_flag once[64];
   static cudaError_t attr_err[64];
   std::call_once(once[d->device], [&] {
@@ -1030,6 +1154,86 @@ struct NoAllocScratch {
 };
 NoAllocScratch g_noalloc[64];
 
+// Quantize X then multiply.  Given activation buffers, the quantize kernel
+// writes (a_codes, a_scales) and the GEMM reads them.  Without them,
+// decode-sized M runs as one kernel whose epilogue warps quantize X into
+// shared memory before the first MMA.  (That one-kernel form measured slower
+// than the two kernels on the decode shape, 15.7 vs 12.9 us: the 148 CTAs
+// each quantize most of X again, in four warps that cannot hide latency,
+// whereas the quantize kernel spreads X over the whole GPU once.)
+constexpr int kLinearMaxM = 32;
+
+bool linear_fused_fits(const DeviceInfo* d, int64_t M, int64_t N, int64_t K) {
+  if (M > kLinearMaxM) return false;
+  const int64_t units = ceil_div(N, kBM) * ceil_div(K, 64 * Cfg<16, true>::kKB);
+  const int64_t grid = units < d->sm_count ? units : d->sm_count;
+  return ceil_div(units, grid) <= Cfg<16, true, 1>::kActSteps;   // steps per CTA, at most
+}
+
+template <int BN, int QX>
+cudaError_t launch_linear(const GemmParams& p, const DeviceInfo* d, cudaStream_t st, bool f32) {
+  return f32 ? launch<BN, true, true, QX>(p, d, st) : launch<BN, true, false, QX>(p, d, st);
+}
+
+nvfp4_status run_linear(const void* x, nvfp4_in_dtype x_dtype, int64_t M, int64_t K, float ga, const uint8_t* w_codes,
+                        const uint8_t* w_scales, float gw, int64_t N, void* out, nvfp4_out_dtype out_dtype,
+                        uint8_t* a_codes, uint8_t* a_scales, cudaStream_t st) {
+  if (!x || !w_codes || !w_scales || !out) return NVFP4_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 32 || K % 32 != 0) return NVFP4_ERR_INVALID_ARG;
+  if (x_dtype != NVFP4_IN_BF16 && x_dtype != NVFP4_IN_F32) return NVFP4_ERR_INVALID_ARG;
+  if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F32) return NVFP4_ERR_INVALID_ARG;
+  if (!finite_positive(ga) || !finite_positive(gw)) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(out)) return NVFP4_ERR_ALIGNMENT;
+  if (M > (1ll << 31) - 256 || N > (1ll << 31) - 256 || K > (1ll << 31)) return NVFP4_ERR_UNSUPPORTED;
+  const DeviceInfo* d = device_info();
+  if (!d) return NVFP4_ERR_CUDA;
+  if (d->major != 10) return NVFP4_ERR_UNSUPPORTED;
+  if ((a_codes && a_scales) || !linear_fused_fits(d, M, N, K)) {
+    if (!a_codes || !a_scales) return NVFP4_ERR_INVALID_ARG;
+    const nvfp4_status s1 = nvfp4_quantize(x, x_dtype, M, K, ga, a_codes, a_scales, NVFP4_SF_TCGEN05, nullptr, st);
+    if (s1 != NVFP4_OK) return s1;
+    return nvfp4_gemm(a_codes, a_scales, ga, w_codes, w_scales, gw, M, N, K, out, out_dtype, st);
+  }
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  Workspace w;
+  const cudaError_t e0 = get_workspace(d, st, &w);
+  if (e0 == cudaErrorNotPermitted) return NVFP4_ERR_UNSUPPORTED;
+  if (e0 != cudaSuccess) return cuda_status(e0);
+  p.ws = w.ws;
+  const int bn = M <= 16 ? 16 : 32;
+  constexpr int kkb = Cfg<16, true>::kKB;
+  p.rows_p = (int)N;
+  p.rows_q = (int)M;
+  p.sf_p = w_scales;
+  p.sf_q = nullptr;
+  if (!make_code_map(&p.tmap_p, w_codes, p.rows_p, K, kBM, 32 * kkb)) return NVFP4_ERR_CUDA;
+  p.tmap_q = p.tmap_p;                      // not read (X is quantized in the kernel)
+  p.out = out;
+  p.tma_store = 0;
+  p.err = d->err_word;
+  p.timeout_ns = wait_timeout_ns();
+  p.M = M;
+  p.N = N;
+  p.rb_q = 1;
+  p.kc = (int)ceil_div(K, 64);
+  p.kt = (int)ceil_div(K, 64 * kkb);
+  p.tiles_p = (int)ceil_div(p.rows_p, kBM);
+  p.tiles_q = 1;
+  p.n_seg = 1;
+  p.seg_end[0] = (int)N;
+  p.seg_alpha[0] = alpha_of(ga, gw);
+  p.x = x;
+  p.x_gs = ga;
+  p.K = K;
+  const bool f32 = out_dtype == NVFP4_OUT_F32;
+  const bool xf32 = x_dtype == NVFP4_IN_F32;
+  cudaError_t e;
+  if (bn == 16) e = xf32 ? launch_linear<16, 2>(p, d, st, f32) : launch_linear<16, 1>(p, d, st, f32);
+  else e = xf32 ? launch_linear<32, 2>(p, d, st, f32) : launch_linear<32, 1>(p, d, st, f32);
+  return cuda_status(e);
+}
+
 }  // namespace
 
 // After a launch whose bounded wait ran out, partial words may be left full;
@@ -1122,6 +1326,13 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float a
   const float gs[1] = {w_global_scale};
   return run_gemm(a_codes, a_scales, a_global_scale, w_codes, w_scales, offs, gs, 1, M, N, K, out, out_dtype,
                   (cudaStream_t)stream);
+}
+
+nvfp4_status nvfp4_linear(const void* x, nvfp4_in_dtype x_dtype, int64_t M, int64_t K, float a_global_scale,
+                          const uint8_t* w_codes, const uint8_t* w_scales, float w_global_scale, int64_t N, void* out,
+                          nvfp4_out_dtype out_dtype, uint8_t* a_codes, uint8_t* a_scales, nvfp4_stream_t stream) {
+  return run_linear(x, x_dtype, M, K, a_global_scale, w_codes, w_scales, w_global_scale, N, out, out_dtype, a_codes,
+                    a_scales, (cudaStream_t)stream);
 }
 
 nvfp4_status nvfp4_fused_proj(const uint8_t* a_codes, const uint8_t* a_scales, float a_global_scale,
