@@ -155,6 +155,20 @@ NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scale
                         int64_t M, int64_t N, int64_t K, void* out, nvfp4_out_dtype out_dtype,
                         nvfp4_stream_t stream);
 
+/* Declare [base, base + bytes) read-only while library calls run (typically
+ * the quantized weights of a model in serving).  No counterpart in the
+ * pages: a scheduling hint.  A GEMM whose weight codes and scales both lie in
+ * declared memory loads its first weight stages before waiting for the
+ * preceding kernel on the stream to finish (programmatic dependent launch),
+ * instead of only prefetching them into L2.  The caller guarantees that no
+ * kernel writes declared memory while a library call that reads it may run;
+ * writing it anyway (for example, quantizing new weights into it just before
+ * a GEMM on the same stream) can make that GEMM read stale weights.
+ * Declarations accumulate until nvfp4_forget_static().
+ * Errors: INVALID_ARG (NULL base or zero bytes). */
+NVFP4_API nvfp4_status nvfp4_declare_static(const void* base, size_t bytes);
+NVFP4_API void nvfp4_forget_static(void);
+
 /* The whole W4A4 linear layer: quantize the activation with a_global_scale
  * (as nvfp4_quantize, TCGEN05 scales) and multiply by the quantized weight
  * (as nvfp4_gemm) [picx.dev summary, "Background": activations and weights

@@ -45,6 +45,9 @@ _lib.nvfp4_amax.argtypes = [_vp, ctypes.c_int, _i64, _i64, _vp, _vp]
 _lib.nvfp4_quantize.argtypes = [_vp, ctypes.c_int, _i64, _i64, _f32, _vp, _vp, ctypes.c_int, _vp, _vp]
 _lib.nvfp4_swizzle_scales.argtypes = [_vp, _i64, _i64, _vp, _vp]
 _lib.nvfp4_gemm.argtypes = [_vp, _vp, _f32, _vp, _vp, _f32, _i64, _i64, _i64, _vp, ctypes.c_int, _vp]
+_lib.nvfp4_declare_static.argtypes = [_vp, ctypes.c_size_t]
+_lib.nvfp4_forget_static.argtypes = []
+_lib.nvfp4_forget_static.restype = None
 _lib.nvfp4_linear.argtypes = [_vp, ctypes.c_int, _i64, _i64, _f32, _vp, _vp, _f32, _i64, _vp, ctypes.c_int, _vp, _vp,
                               _vp]
 _lib.nvfp4_gemm_noalloc.argtypes = [_vp, _vp, _f32, _vp, _vp, _f32, _i64, _i64, _i64, _vp, ctypes.c_int, _vp]
@@ -149,6 +152,14 @@ def nvfp4_gemm(a_codes, a_scales, a_global_scale, w_codes, w_scales, w_global_sc
     _check("nvfp4_gemm", _lib.nvfp4_gemm(_ptr(a_codes), _ptr(a_scales), float(a_global_scale), _ptr(w_codes),
                                          _ptr(w_scales), float(w_global_scale), M, N, K, _ptr(out),
                                          _out_dtype(out), _stream(out)))
+
+
+def nvfp4_declare_static(t: torch.Tensor) -> None:
+    _check("nvfp4_declare_static", _lib.nvfp4_declare_static(_ptr(t), t.numel() * t.element_size()))
+
+
+def nvfp4_forget_static() -> None:
+    _lib.nvfp4_forget_static()
 
 
 def nvfp4_linear(x: torch.Tensor, a_global_scale, w_codes, w_scales, w_global_scale, N, out: torch.Tensor,

@@ -38,6 +38,7 @@
 #include <map>
 #include <mutex>
 #include <utility>
+#include <vector>
 
 #include "block_quant.cuh"
 #include "common.h"
@@ -69,6 +70,7 @@ struct alignas(64) GemmParams {
   int kt;                // ceil(K / (64 * kKB)): pipeline steps per tile
   int tiles_p, tiles_q;
   int tma_store;         // 1: output through shared memory and TMA stores
+  int w_static;          // 1: the weight lies in memory declared read-only (nvfp4_declare_static)
   int n_seg;
   int seg_end[NVFP4_MAX_SEGMENTS];
   float seg_alpha[NVFP4_MAX_SEGMENTS];
@@ -372,22 +374,40 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX>::kThreads, 1)
       const WorkIter w0 = work_begin(p, SWAP);
       // prologue: the first kStages stages are free
       int npro = 0;
+      const bool w_static = p.w_static != 0;
       for_steps(w0, 0, C::kStages, [&](int j, int p0, int q0, int k) {
-        const uint32_t sf_bytes = (uint32_t)min(C::kKB, kc - C::kKB * k) * kSfChunk;
-        if (SWAP) {
-          tma_prefetch_l2_2d(&p.tmap_p, k * C::kRowBytes, p0);
-          bulk_prefetch_l2(p.sf_p + ((size_t)(p0 >> 7) * kc + C::kKB * k) * kSfChunk, sf_bytes);
+        if (w_static) {
+          // a weight declared read-only cannot be written by the preceding
+          // kernel: load its first stages now
+          expect(j, q0, k);
+          if (SWAP) load_p(j, p0, k);
+          else load_q(j, q0, k);
+          issued_mask |= 1u << j;
         } else {
-          tma_prefetch_l2_2d(&p.tmap_q, k * C::kRowBytes, q0);
+          const uint32_t sf_bytes = (uint32_t)min(C::kKB, kc - C::kKB * k) * kSfChunk;
+          if (SWAP) {
+            tma_prefetch_l2_2d(&p.tmap_p, k * C::kRowBytes, p0);
+            bulk_prefetch_l2(p.sf_p + ((size_t)(p0 >> 7) * kc + C::kKB * k) * kSfChunk, sf_bytes);
+          } else {
+            tma_prefetch_l2_2d(&p.tmap_q, k * C::kRowBytes, q0);
+          }
         }
         npro = j + 1;
       });
       asm volatile("griddepcontrol.wait;" ::: "memory");
       for_steps(w0, 0, npro, [&](int j, int p0, int q0, int k) {
-        expect(j, q0, k);
-        load_p(j, p0, k);
-        if (!C::kQx) load_q(j, q0, k);
-        issued_mask |= 1u << j;
+        if (w_static) {
+          if (SWAP) {
+            if (!C::kQx) load_q(j, q0, k);
+          } else {
+            load_p(j, p0, k);
+          }
+        } else {
+          expect(j, q0, k);
+          load_p(j, p0, k);
+          if (!C::kQx) load_q(j, q0, k);
+          issued_mask |= 1u << j;
+        }
       });
       int stage = npro % C::kStages;
       uint32_t phase = npro == C::kStages ? 1u : 0u;
@@ -987,6 +1007,20 @@ bool make_out_map(CUtensorMap* m, void* base, int64_t M, int64_t N, bool f32) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Memory the caller declared read-only for the duration of library calls
+// (nvfp4_declare_static): a GEMM whose weight codes and scales lie inside it
+// loads its first weight stages before waiting on the preceding kernel.
+std::mutex g_static_mu;
+std::vector<std::pair<uintptr_t, uintptr_t>> g_static_ranges;   // [begin, end)
+
+bool is_static(const void* p, size_t bytes) {
+  const uintptr_t b = reinterpret_cast<uintptr_t>(p), e = b + bytes;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  for (const auto& r : g_static_ranges)
+    if (b >= r.first && e <= r.second) return true;
+  return false;
+}
+
 // Swapped (decode) tiles are split over the CTAs along K; partial tiles are
 // exchanged through a workspace the library owns: one per (device, stream),
 // allocated (all words empty) on the first swapped call on that stream, kept
@@ -1100,6 +1134,9 @@ nvfp4_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float ga,
   // TMA stores need 16-byte aligned output rows
   const bool f32 = out_dtype == NVFP4_OUT_F32;
   p.tma_store = (!swap && (N * (f32 ? 4 : 2)) % 16 == 0) ? 1 : 0;
+  p.w_static = is_static(w_codes, (size_t)N * (size_t)(K / 2)) &&
+                       is_static(w_scales, nvfp4_scale_bytes(N, K, NVFP4_SF_TCGEN05))
+                   ? 1 : 0;
   if (p.tma_store && !make_out_map(&p.tmap_out, out, M, N, f32)) return NVFP4_ERR_CUDA;
   p.err = d->err_word;
   p.timeout_ns = wait_timeout_ns();
@@ -1209,6 +1246,9 @@ nvfp4_status run_linear(const void* x, nvfp4_in_dtype x_dtype, int64_t M, int64_
   p.sf_q = nullptr;
   if (!make_code_map(&p.tmap_p, w_codes, p.rows_p, K, kBM, 32 * kkb)) return NVFP4_ERR_CUDA;
   p.tmap_q = p.tmap_p;                      // not read (X is quantized in the kernel)
+  p.w_static = is_static(w_codes, (size_t)N * (size_t)(K / 2)) &&
+                       is_static(w_scales, nvfp4_scale_bytes(N, K, NVFP4_SF_TCGEN05))
+                   ? 1 : 0;
   p.out = out;
   p.tma_store = 0;
   p.err = d->err_word;
@@ -1326,6 +1366,19 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float a
   const float gs[1] = {w_global_scale};
   return run_gemm(a_codes, a_scales, a_global_scale, w_codes, w_scales, offs, gs, 1, M, N, K, out, out_dtype,
                   (cudaStream_t)stream);
+}
+
+nvfp4_status nvfp4_declare_static(const void* base, size_t bytes) {
+  if (!base || bytes == 0) return NVFP4_ERR_INVALID_ARG;
+  const uintptr_t b = reinterpret_cast<uintptr_t>(base);
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  g_static_ranges.emplace_back(b, b + bytes);
+  return NVFP4_OK;
+}
+
+void nvfp4_forget_static(void) {
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  g_static_ranges.clear();
 }
 
 nvfp4_status nvfp4_linear(const void* x, nvfp4_in_dtype x_dtype, int64_t M, int64_t K, float a_global_scale,

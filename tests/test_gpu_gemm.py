@@ -226,3 +226,28 @@ def test_gemm_right_after_the_kernel_that_writes_its_operands(M, N, K):
         assert_gemm_close(out.cpu().numpy(), ref, f"{M}x{N}x{K}")
         del wcd, wsd, acd, asd
     check_device_error_word()
+
+
+@pytest.mark.parametrize("M,N,K", [(8, 12288, 5120), (512, 2048, 5120), (3, 200, 96)])
+def test_static_weights_give_the_same_result(M, N, K):
+    # weights declared read-only are loaded before the preceding kernel ends;
+    # the arithmetic is unchanged, so results are bitwise those of the
+    # default path, also when the GEMMs follow each other and the quantizer
+    # back to back
+    (ac, asc, ga), (wc, wsc, gw) = _operands(M, N, K, seed=77)
+    a_d, as_d = to_dev_operand(ac, asc, K)
+    w_d, ws_d = to_dev_operand(wc, wsc, K)
+    x = synth.student_t_outliers(M, K, seed=78, dtype=torch.float32).to(DEV)
+    ref = gpu_gemm(a_d, as_d, ga, w_d, ws_d, gw, M, N, K, torch.float32)
+    nv.nvfp4_declare_static(w_d)
+    nv.nvfp4_declare_static(ws_d)
+    try:
+        outs = []
+        for _ in range(3):
+            qa, qs, _ = gpu_quantize(x, ga)              # a kernel just before, as in a decode step
+            outs.append(gpu_gemm(a_d, as_d, ga, w_d, ws_d, gw, M, N, K, torch.float32))
+        torch.cuda.synchronize()
+    finally:
+        nv.nvfp4_forget_static()
+    assert all(torch.equal(o, ref) for o in outs)
+    check_device_error_word()
