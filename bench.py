@@ -52,7 +52,7 @@ def load_peaks():
 
 def source_hash() -> str:
     h = hashlib.sha256()
-    for name in ("gemm.cu", "quantize.cu", "ptx.cuh", "common.h", "runtime.cu"):
+    for name in ("gemm.cu", "quantize.cu", "block_quant.cuh", "ptx.cuh", "common.h", "runtime.cu"):
         with open(os.path.join(ROOT, "nvfp4_w4a4_quantized_10_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
