@@ -49,7 +49,7 @@ namespace nvfp4 {
 constexpr int kBM = 128;          // MMA M: rows of operand P per tile
 constexpr int kSfChunk = 512;     // bytes of one 128-row x 4-scale chunk
 constexpr int kTmemCols = 512;
-constexpr int kGroupP = 8;        // tile raster: 8 P-tiles share a Q-tile
+constexpr int kGroupP = 64;       // tile raster: 64 P-tiles (8192 rows) share each Q-tile sweep
 constexpr int kStageOutBytes = 16384;   // one 128-row x 128-byte output sub-tile
 constexpr int kEpiBar = 1;        // named barrier id of the 128 epilogue threads
 
