@@ -181,13 +181,6 @@ class Decode:
         self.layer_bytes = M * K * 2 + N * K // 2 + N * K // 16 + M * N * 2
         self.launches_per_step = 2
 
-    def step(self, i):
-        nv = self.nv
-        w = self.w
-        wc, ws = self.w_copies[i % self.n_copies]
-        nv.nvfp4_quantize(self.x, self.ga, self.a_codes, self.a_sc)
-        nv.nvfp4_gemm(self.a_codes, self.a_sc, self.ga, wc, ws, self.gw, w.M, w.N, w.K, self.out)
-
     def gemm_only(self, i):
         w = self.w
         wc, ws = self.w_copies[i % self.n_copies]

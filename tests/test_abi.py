@@ -107,6 +107,34 @@ def test_other_validation():
     assert L.nvfp4_test_wait_timeout(11_000_000_000, None) == nv.ERR_INVALID_ARG
 
 
+def lin(x=A16, dt=0, M=8, K=64, ga=1.0, w=A16, sw=A16, gw=1.0, N=64, out=A16, od=0, ac=None, asc=None):
+    return nv.lib().nvfp4_linear(x, dt, M, K, ctypes.c_float(ga), w, sw, ctypes.c_float(gw), N, out, od, ac, asc,
+                                 None)
+
+
+def test_linear_validation():
+    assert lin(x=None) == nv.ERR_INVALID_ARG
+    assert lin(w=None) == nv.ERR_INVALID_ARG
+    assert lin(out=None) == nv.ERR_INVALID_ARG
+    assert lin(M=0) == nv.ERR_INVALID_ARG
+    assert lin(N=0) == nv.ERR_INVALID_ARG
+    assert lin(K=48) == nv.ERR_INVALID_ARG
+    assert lin(dt=3) == nv.ERR_INVALID_ARG
+    assert lin(od=3) == nv.ERR_INVALID_ARG
+    assert lin(ga=float("inf")) == nv.ERR_INVALID_ARG
+    assert lin(gw=0.0) == nv.ERR_INVALID_ARG
+    assert lin(x=A1) == nv.ERR_ALIGNMENT
+    assert lin(sw=A1) == nv.ERR_ALIGNMENT
+
+
+def test_declare_static_validation():
+    L = nv.lib()
+    assert L.nvfp4_declare_static(None, 64) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_declare_static(A16, 0) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_declare_static(A16, 64) == nv.OK
+    L.nvfp4_forget_static()
+
+
 def test_product_package_does_not_import_the_oracle():
     import pathlib
     pkg = pathlib.Path(nv.__file__).parent
