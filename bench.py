@@ -51,10 +51,15 @@ def load_peaks():
 
 
 def source_hash() -> str:
+    """Hash of the library's kernel sources with // comments and blank lines
+    removed, so that a comment edit keeps recorded counters valid."""
     h = hashlib.sha256()
     for name in ("gemm.cu", "quantize.cu", "block_quant.cuh", "ptx.cuh", "common.h", "runtime.cu"):
-        with open(os.path.join(ROOT, "nvfp4_w4a4_quantized_10_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "nvfp4_w4a4_quantized_10_b200", "csrc", name), encoding="utf-8") as f:
+            for line in f:
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

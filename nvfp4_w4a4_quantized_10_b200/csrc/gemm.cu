@@ -9,25 +9,30 @@
 //   out[m,n] = alpha(n) * sum_b sA[m,b] sW[n,b] sum_{k in b} e2m1(A[m,k]) e2m1(W[n,k])
 //   alpha(n) = 1 / (gA * gW[segment of n])
 //
-// Design (one persistent CTA per SM, 6 warps):
+// Design (one persistent CTA per SM):
 //   warp 0    TMA producer: per 256-wide K step, one 2-D TMA box of each
 //             operand's codes (128-byte rows, 128B swizzle) and one or two
 //             bulk copies of the pre-swizzled E4M3 scale chunks, all landing
 //             on one mbarrier with an expected byte count.
-//   warp 1    TMEM allocator and MMA issuer: copies the scale chunks from
-//             shared memory into TMEM (tcgen05.cp 32x128b.warpx4), then
-//             issues four tcgen05.mma kind::mxf4nvf4 block_scale (K = 64
-//             each) into the FP32 accumulator in TMEM, and releases the
-//             stage with tcgen05.commit.
+//   warp 1    TMEM allocator and MMA issuer: per step, four tcgen05.mma
+//             kind::mxf4nvf4 block_scale (K = 64 each) into the FP32
+//             accumulator in TMEM, then tcgen05.commit to release the stage.
 //   warps 2-5 epilogue: tcgen05.ld the accumulator (one TMEM lane per
 //             output row), scale by alpha, round once to bf16 (or keep
-//             f32), free the accumulator, store.
+//             f32), free the accumulator, store.  With an in-kernel
+//             activation (nvfp4_linear) they first quantize X into shared
+//             memory.
+//   warps 6+  scale copies: one warp for P's scale chunks and one per
+//             128-row block of Q's move each step's scales into TMEM
+//             (tcgen05.cp 32x128b.warpx4) and signal the MMA warp.  Each
+//             tcgen05 instruction holds its issuing thread for tens of
+//             cycles; spread over warps, copies and MMAs overlap.
 // Two tile shapes:
 //   normal  P = activations (128-row tiles), Q = weight (256-row tiles):
 //           prefill and fused projections.
 //   swap    P = weight (128-row tiles), Q = all activation rows (<= 128):
-//           decode, so the 128-row MMA dimension walks the weight and the
-//           grid covers N/128 tiles that stream W from HBM.
+//           decode, so the 128-row MMA dimension walks the weight; the
+//           K loop is split over the CTAs (stream-K) so every SM streams W.
 // Every mbarrier wait is bounded (see ptx.cuh); on timeout the CTA drains
 // its in-flight copies and MMAs (bounded again), frees TMEM and exits.
 #include <cuda.h>
