@@ -55,6 +55,9 @@ def lib():
         L.orc_fused_proj.argtypes = [u8p, u8p, ctypes.c_float, u8p, u8p, i64p, f32p,
                                      ctypes.c_int, i64, i64, f64p]
         L.orc_gemm_exact.argtypes = [u8p, u8p, u8p, u8p, i64, i64, i64, i64p]
+        L.orc_saturation.argtypes = [f32p, i64, i64, ctypes.c_float, i64p]
+        L.orc_harmonize_scales.argtypes = [u8p, i64, i64, i64p, f32p, ctypes.c_int,
+                                           ctypes.c_float, u8p]
         L.orc_set_threads.argtypes = [ctypes.c_int]
         L.orc_get_threads.restype = ctypes.c_int
         _lib = L
@@ -204,3 +207,39 @@ def gemm_exact(a_codes, a_scales, w_codes, w_scales):
                          _p(w_codes, ctypes.c_uint8), _p(w_scales, ctypes.c_uint8),
                          M, N, K, _p(S, ctypes.c_int64))
     return S
+
+
+# ---- static calibration and offline harmonisation ------------------------
+
+def calibrate_amax(batches) -> np.float32:
+    """Largest magnitude over several calibration batches: the running maximum
+    of the per-batch amax, the statistic a static global scale is built from
+    (anthology record LIT-800, "Key takeaways": calibration-only recipe)."""
+    m = np.float32(0.0)
+    for b in batches:
+        m = max(m, amax(b))
+    return np.float32(m)
+
+
+def saturation(x, g):
+    """(blocks with a clipped scale, elements with a clipped code, blocks whose
+    scale underflowed to zero) when x is quantized with global scale g."""
+    x = _c(x, np.float32)
+    M, K = x.shape
+    counts = np.zeros(3, np.int64)
+    lib().orc_saturation(_p(x, ctypes.c_float), M, K, float(np.float32(g)), _p(counts, ctypes.c_int64))
+    return tuple(int(c) for c in counts)
+
+
+def harmonize_scales(scales, seg_offsets, seg_gs, g):
+    """Row-major block scales [R, K/16] of a fused weight rewritten from
+    per-segment global scales seg_gs to one common scale g (codes unchanged)."""
+    scales = _c(scales, np.uint8)
+    R, nb = scales.shape
+    offs = _c(seg_offsets, np.int64)
+    gs = _c(seg_gs, np.float32)
+    out = np.empty_like(scales)
+    lib().orc_harmonize_scales(_p(scales, ctypes.c_uint8), R, nb * 16, _p(offs, ctypes.c_int64),
+                               _p(gs, ctypes.c_float), len(gs), float(np.float32(g)),
+                               _p(out, ctypes.c_uint8))
+    return out

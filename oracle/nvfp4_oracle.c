@@ -374,3 +374,78 @@ void orc_gemm_exact(const uint8_t* a_codes, const uint8_t* a_scales,
             S[m * N + n] = acc;
         }
 }
+
+/* ------------------------------------------------------------------ */
+/* Static calibration: how much a fixed global scale clips (R15)       */
+/* ------------------------------------------------------------------ */
+
+/* A global scale calibrated on other data can be too large for a new input:
+ * a block's scale target t = (amax_b / 6) * g then exceeds 448 and the E4M3
+ * scale saturates, after which x * r can exceed 6 and the E2M1 code
+ * saturates too.  [anthology record LIT-800, "Key takeaways": the recipe is
+ * calibration-only, on a fixed set of sequences; cctest.ai article,
+ * "Introduction"]  The arithmetic is that of orc_quantize, step for step.
+ *   counts[0] = blocks with t > 448 (scale clipped)
+ *   counts[1] = elements with |x * r| > 6 (code clipped)
+ *   counts[2] = blocks whose scale rounded to zero while amax_b > 0 */
+void orc_saturation(const float* x, int64_t M, int64_t K, float g, int64_t* counts) {
+    const int64_t nb = K / 16;
+    int64_t c0 = 0, c1 = 0, c2 = 0;
+#pragma omp parallel for schedule(static) reduction(+ : c0, c1, c2)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t b = 0; b < nb; ++b) {
+            const float* xb = x + m * K + b * 16;
+            float amax = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                float a = fabsf(xb[i]);
+                if (a > amax) amax = a;
+            }
+            float q = amax / 6.0f;
+            float t = q * g;
+            if (t > 448.0f) c0 += 1;
+            uint8_t s = orc_e4m3_encode(t);
+            if ((s & 0x7F) == 0) {
+                if (amax > 0.0f) c2 += 1;
+                continue;
+            }
+            float r = g / (float)orc_e4m3_decode(s);
+            for (int i = 0; i < 16; ++i) {
+                float y = xb[i] * r;
+                if (fabsf(y) > 6.0f) c1 += 1;
+            }
+        }
+    }
+    counts[0] = c0;
+    counts[1] = c1;
+    counts[2] = c2;
+}
+
+/* ------------------------------------------------------------------ */
+/* Offline global-scale harmonisation of a fused weight (R14)          */
+/* ------------------------------------------------------------------ */
+
+/* A fused projection weight stacks row segments [offs[i], offs[i+1]), each
+ * quantized with its own global scale gs[i].  A kernel that applies one
+ * scale to the whole GEMM needs the checkpoint rewritten to a common scale g
+ * first ("pre-harmonized") [cctest.ai article, "Main findings"; anthology
+ * record LIT-800, "Standing in the anthology"].  The element codes are kept;
+ * every block scale s of segment i becomes
+ *     s' = E4M3(e4m3(s) * q_i),   q_i = g / gs[i]
+ * with q_i rounded to FP32 once per segment and one FP32 multiply per scale,
+ * so that e2m1 * e4m3(s') / g approximates e2m1 * e4m3(s) / gs[i].
+ * scales and out are [R, K/16] row-major; rows outside every segment are
+ * copied unchanged. */
+void orc_harmonize_scales(const uint8_t* scales, int64_t R, int64_t K, const int64_t* offs,
+                          const float* gs, int nseg, float g, uint8_t* out) {
+    const int64_t nb = K / 16;
+    memcpy(out, scales, (size_t)(R * nb));
+    for (int i = 0; i < nseg; ++i) {
+        float qi = g / gs[i];
+        for (int64_t r = offs[i]; r < offs[i + 1] && r < R; ++r)
+            for (int64_t j = 0; j < nb; ++j) {
+                float sv = (float)orc_e4m3_decode(scales[r * nb + j]);
+                float y = sv * qi;
+                out[r * nb + j] = orc_e4m3_encode(y);
+            }
+    }
+}
