@@ -50,16 +50,28 @@ def load_peaks():
         return FALLBACK_PEAKS, "fallback"
 
 
-def source_hash() -> str:
-    """Hash of the library's kernel sources with // comments and blank lines
-    removed, so that a comment edit keeps recorded counters valid."""
+# The sources each kernel's recorded counters depend on.
+KERNEL_SOURCES = {
+    "nvfp4_gemm_kernel": ("gemm.cu", "block_quant.cuh", "ptx.cuh", "common.h", "runtime.cu"),
+    "quantize_kernel": ("quantize.cu", "block_quant.cuh", "ptx.cuh", "common.h"),
+}
+
+
+def source_hash(kernel: str, read=None) -> str:
+    """Hash of one kernel's sources with // comments and blank lines removed,
+    so that a comment edit, or a change to another kernel, keeps its recorded
+    counters valid.  read(name) -> text overrides reading the working tree."""
     h = hashlib.sha256()
-    for name in ("gemm.cu", "quantize.cu", "block_quant.cuh", "ptx.cuh", "common.h", "runtime.cu"):
-        with open(os.path.join(ROOT, "nvfp4_w4a4_quantized_10_b200", "csrc", name), encoding="utf-8") as f:
-            for line in f:
-                code = line.split("//", 1)[0].rstrip()
-                if code:
-                    h.update(code.encode() + b"\n")
+    for name in KERNEL_SOURCES[kernel]:
+        if read is None:
+            with open(os.path.join(ROOT, "nvfp4_w4a4_quantized_10_b200", "csrc", name), encoding="utf-8") as f:
+                text = f.read()
+        else:
+            text = read(name)
+        for line in text.splitlines():
+            code = line.split("//", 1)[0].rstrip()
+            if code:
+                h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 
@@ -71,7 +83,7 @@ def profiled_traffic(kernel: str, workload: str):
         with open(path) as f:
             t = json.load(f)
         e = t[f"{kernel}:{workload}"]
-        if e.get("source_hash") == source_hash():
+        if e.get("source_hash") == source_hash(kernel):
             return e["dram_bytes_per_launch"]
     except Exception:
         pass
@@ -555,13 +567,115 @@ def measure_quant_sweep(torch, nv, synth, dev, args, stream, peaks):
     return sweep
 
 
+def measure_calibration(torch, nv, synth, dev, args, stream, peaks):
+    """Static calibration: running amax over the calibration batches (one pass
+    = CALIB_BATCHES batches), then the static-scale quantization of a held-out
+    batch with larger outliers.  Two alternating batch sets and four held-out
+    copies keep every pass's inputs out of L2."""
+    hbm_peak = float(peaks["hbm_gbs"])
+    M, K, nb = synth.CALIB_M, synth.CALIB_K, synth.CALIB_BATCHES
+    sets = [[synth.calibration_batch(i + nb * j, M, K, device=dev) for i in range(nb)] for j in range(2)]
+    run = torch.empty(2, dtype=torch.float32, device=dev)
+
+    def amax_pass(i):
+        r = run[i % 2:i % 2 + 1]
+        nv.nvfp4_amax(sets[i % 2][0], r)
+        for b in sets[i % 2][1:]:
+            nv.nvfp4_amax_accumulate(b, r)
+
+    kk = max(3, min(args.steps, 50))
+    with torch.cuda.stream(stream):
+        ms_a, g1 = time_graph(torch, amax_pass, kk, 3, stream)
+    del g1
+    torch.cuda.synchronize()
+    g_static = 2688.0 / float(run[0].item())
+    held = synth.held_out_batch(M, K, device=dev)
+    copies = [held] + [held.clone() for _ in range(3)]
+    codes, sc = nv.alloc_quantized(M, K, dev)
+
+    def quant(i):
+        nv.nvfp4_quantize(copies[i % 4], g_static, codes, sc)
+
+    with torch.cuda.stream(stream):
+        ms_q, g2 = time_graph(torch, quant, kk, 3, stream)
+    del g2
+    torch.cuda.synchronize()
+    held_sat = int((sc == 0x7E).sum().item())
+    cal_codes, cal_sc = nv.alloc_quantized(M, K, dev)
+    nv.nvfp4_quantize(sets[0][0], g_static, cal_codes, cal_sc)
+    torch.cuda.synchronize()
+    cal_sat = int((cal_sc == 0x7E).sum().item())
+    pass_bytes = nb * M * K * 2
+    q_bytes = M * K * 2 + M * K // 2 + M * K // 16
+    res = {"workload": f"{nb} calibration batches X[{M},{K}] bf16 (outliers 48x RMS), then a held-out "
+                       f"batch (368x RMS) quantized with the static scale",
+           "amax_pass_us": ms_a * 1e3, "amax_GB/s": pass_bytes / (ms_a * 1e-3) / 1e9,
+           "amax_frac_hbm": pass_bytes / (ms_a * 1e-3) / 1e9 / hbm_peak,
+           "static_quant_us": ms_q * 1e3, "static_quant_GB/s": q_bytes / (ms_q * 1e-3) / 1e9,
+           "static_quant_frac_hbm": q_bytes / (ms_q * 1e-3) / 1e9 / hbm_peak,
+           "scale_bytes_at_448": {"held_out": held_sat, "calibration_batch_0": cal_sat},
+           "launches_per_pass": nb}
+    del sets, copies, codes, sc
+    return res
+
+
+def measure_harmonize(torch, nv, synth, dev, rank, l2, args, stream, peaks):
+    """Offline scale harmonisation of the fused GDN weight (TCGEN05 scales)
+    to g = min g_i, timed over enough scale copies to exceed L2; then the
+    single-scale GEMM on the harmonized scales and the unrepaired single-
+    scale GEMM, each compared per segment with the exact per-segment
+    epilogue (relative Frobenius error)."""
+    hbm_peak = float(peaks["hbm_gbs"])
+    f = FusedGDN(torch, nv, synth, dev, rank, l2)
+    w = f.w
+    g = min(f.gs)
+    n_bytes = f.ws.numel()
+    n_copies = max(2, math.ceil(3 * l2 / (2 * n_bytes)))
+    srcs = [f.ws] + [f.ws.clone() for _ in range(n_copies - 1)]
+    dsts = [torch.empty_like(f.ws) for _ in range(n_copies)]
+
+    def harm(i):
+        nv.nvfp4_harmonize_scales(srcs[i % n_copies], w.N, w.K, f.offs, f.gs, g, dsts[i % n_copies])
+
+    kk = max(3, min(args.steps, 50))
+    with torch.cuda.stream(stream):
+        ms_h, g1 = time_graph(torch, harm, kk, 3, stream)
+    del g1
+    f.step(0)
+    exact = torch.empty(w.M, w.N, dtype=torch.float32, device=dev)
+    nv.nvfp4_fused_proj(f.a_codes, f.a_sc, f.ga, f.wc, f.ws, f.offs, f.gs, w.M, w.K, exact)
+    harmonized = torch.empty_like(exact)
+    nv.nvfp4_gemm(f.a_codes, f.a_sc, f.ga, f.wc, dsts[0], g, w.M, w.N, w.K, harmonized)
+    single = torch.empty_like(exact)
+    nv.nvfp4_gemm(f.a_codes, f.a_sc, f.ga, f.wc, f.ws, f.gs[0], w.M, w.N, w.K, single)
+    torch.cuda.synchronize()
+
+    def seg_err(o):
+        out = []
+        for i in range(len(f.gs)):
+            a, b = o[:, f.offs[i]:f.offs[i + 1]].double(), exact[:, f.offs[i]:f.offs[i + 1]].double()
+            out.append(float((a - b).norm() / b.norm()))
+        return out
+
+    byts = 2 * n_bytes
+    res = {"workload": f"fused GDN weight scales [{w.N}, {w.K // 16}] TCGEN05 ({n_bytes} B), segments "
+                       f"{list(w.segments)}, to g = min g_i",
+           "us": ms_h * 1e3, "GB/s": byts / (ms_h * 1e-3) / 1e9, "frac_hbm": byts / (ms_h * 1e-3) / 1e9 / hbm_peak,
+           "g_ratio": [g / x for x in f.gs],
+           "seg_rel_fro_harmonized": seg_err(harmonized),
+           "seg_rel_fro_single_scale_unrepaired": seg_err(single)}
+    del f, srcs, dsts
+    nv.nvfp4_forget_static()
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--only", default="all", choices=["all", "decode", "prefill", "fused", "quant"])
+    ap.add_argument("--only", default="all", choices=["all", "decode", "prefill", "fused", "quant", "calib", "harmonize"])
     ap.add_argument("--prefill-m", type=int, default=0, help="override M of the prefill workload")
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed decode steps first")
     ap.add_argument("--no-extra", action="store_true")
@@ -611,6 +725,10 @@ def main():
             res = measure_prefill(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind)
         elif args.only == "fused":
             res = measure_fused(torch, nv, synth, dev, rank, l2, args, stream)
+        elif args.only == "calib":
+            res = measure_calibration(torch, nv, synth, dev, args, stream, peaks)
+        elif args.only == "harmonize":
+            res = measure_harmonize(torch, nv, synth, dev, rank, l2, args, stream, peaks)
         else:
             res = measure_quant_sweep(torch, nv, synth, dev, args, stream, peaks)
         sampler.stop()
@@ -625,6 +743,8 @@ def main():
             "prefill": measure_prefill(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind),
             "fused_gdn": measure_fused(torch, nv, synth, dev, rank, l2, args, stream),
             "quantize_sweep": measure_quant_sweep(torch, nv, synth, dev, args, stream, peaks),
+            "static_calibration": measure_calibration(torch, nv, synth, dev, args, stream, peaks),
+            "harmonize": measure_harmonize(torch, nv, synth, dev, rank, l2, args, stream, peaks),
         }
     sampler.stop()
     if clk is not None:

@@ -103,6 +103,21 @@ NVFP4_API size_t nvfp4_scale_bytes(int64_t rows, int64_t K, nvfp4_sf_layout layo
 NVFP4_API nvfp4_status nvfp4_amax(const void* x, nvfp4_in_dtype dtype, int64_t M, int64_t K,
                         float* amax_out, nvfp4_stream_t stream);
 
+/* Running per-tensor amax over calibration batches: the statistic a static
+ * activation scale g = 448*6/amax is built from, where the scale is fixed
+ * once from calibration data and then serves every later input
+ * [anthology record LIT-800, "Key takeaways": calibration-only recipe;
+ * cctest.ai article, "Introduction"].
+ *   x            device, [M, K] row-major, bf16 or f32 per `dtype`, 16-B aligned
+ *   running_amax device, one float holding +0 or a positive finite value (set
+ *                it to 0 before the first batch); replaced by
+ *                max(running_amax, max |x|).  Nothing is reset: call once per
+ *                batch on one stream, then read the float back.
+ * Errors: INVALID_ARG (null, M < 1, K < 1, M*K*element size not a multiple
+ * of 16 bytes), ALIGNMENT, CUDA. */
+NVFP4_API nvfp4_status nvfp4_amax_accumulate(const void* x, nvfp4_in_dtype dtype, int64_t M, int64_t K,
+                                   float* running_amax, nvfp4_stream_t stream);
+
 /* NVFP4 quantization of X [M, K] with a given FP32 global scale
  * [picx.dev summary, "Background"].  For each block of 16 elements along K:
  *   amax_b = max |x|;  t = (amax_b / 6) * g  (FP32, in this order);
@@ -237,6 +252,32 @@ NVFP4_API nvfp4_status nvfp4_fused_proj(const uint8_t* a_codes, const uint8_t* a
                               const int64_t* seg_offsets, const float* seg_global_scales, int n_seg,
                               int64_t M, int64_t K, void* out, nvfp4_out_dtype out_dtype,
                               nvfp4_stream_t stream);
+
+/* Offline global-scale harmonisation of a fused weight: segments quantized
+ * with their own global scales g_i are rewritten to one common scale g, so a
+ * kernel that applies a single scale to the whole fused GEMM serves them
+ * correctly ("pre-harmonized" checkpoint) [cctest.ai article, "Main
+ * findings"; anthology record LIT-800, "Standing in the anthology": per-module
+ * scales served by a fused kernel give mis-scaled gates].  The E2M1 codes are
+ * kept; every block scale s of a row in segment i becomes
+ *     s' = E4M3(e4m3(s) * q_i),  q_i = g / g_i  (FP32, rounded once per segment)
+ * with nearest-even rounding and saturation at 448.  g = min g_i keeps every
+ * q_i <= 1, so nothing saturates; the dequantized weights then move by at most
+ * half an E4M3 step (more where s' falls into the E4M3 subnormal range).
+ *   scales   device, nvfp4_scale_bytes(N, K, layout) bytes, 16-byte aligned
+ *   layout   layout of both scales and out (row-major [N, K/16] or TCGEN05)
+ *   seg_offsets        host int64[n_seg + 1]: 0 = o_0 < o_1 < ... < o_n <= N;
+ *                      rows from o_n to N are copied unchanged
+ *   seg_global_scales  host float[n_seg] (g_i), each finite and > 0
+ *   common_global_scale  g, finite and > 0
+ *   out      device, same size and layout as scales, 16-byte aligned; may equal
+ *            scales (in place); any other overlap is undefined.  NaN scale
+ *            bytes (0x7F, 0xFF) give unspecified bytes.
+ * Errors: INVALID_ARG (null, N < 1, K < 16 or K % 16, bad layout, bad
+ * segments or scales), ALIGNMENT, CUDA. */
+NVFP4_API nvfp4_status nvfp4_harmonize_scales(const uint8_t* scales, int64_t N, int64_t K, nvfp4_sf_layout layout,
+                                    const int64_t* seg_offsets, const float* seg_global_scales, int n_seg,
+                                    float common_global_scale, uint8_t* out, nvfp4_stream_t stream);
 
 /* Element conversions exactly as the quantizer performs them, exposed so the
  * encoders can be checked exhaustively.

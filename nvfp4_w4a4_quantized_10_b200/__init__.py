@@ -7,7 +7,7 @@ on a non-OK status.  All quantization and GEMM work runs in the library's
 CUDA kernels; there is no CPU fallback.  PyTorch supplies device memory and
 streams.
 
-The library is built in-tree by ``python -m nvfp4_w4a4_quantized_10_b200.build``;
+The library is built in-tree by ``python nvfp4_w4a4_quantized_10_b200/build.py``;
 importing this package without it raises ImportError.
 """
 from __future__ import annotations
@@ -24,7 +24,7 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "nvfp4.h")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"libnvfp4.so is not built ({LIB_PATH}); run "
-                      "`python -m nvfp4_w4a4_quantized_10_b200.build`")
+                      "`python nvfp4_w4a4_quantized_10_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -42,6 +42,9 @@ _f32 = ctypes.c_float
 _lib.nvfp4_scale_bytes.restype = ctypes.c_size_t
 _lib.nvfp4_scale_bytes.argtypes = [_i64, _i64, ctypes.c_int]
 _lib.nvfp4_amax.argtypes = [_vp, ctypes.c_int, _i64, _i64, _vp, _vp]
+_lib.nvfp4_amax_accumulate.argtypes = [_vp, ctypes.c_int, _i64, _i64, _vp, _vp]
+_lib.nvfp4_harmonize_scales.argtypes = [_vp, _i64, _i64, ctypes.c_int, ctypes.POINTER(_i64), ctypes.POINTER(_f32),
+                                        ctypes.c_int, _f32, _vp, _vp]
 _lib.nvfp4_quantize.argtypes = [_vp, ctypes.c_int, _i64, _i64, _f32, _vp, _vp, ctypes.c_int, _vp, _vp]
 _lib.nvfp4_swizzle_scales.argtypes = [_vp, _i64, _i64, _vp, _vp]
 _lib.nvfp4_gemm.argtypes = [_vp, _vp, _f32, _vp, _vp, _f32, _i64, _i64, _i64, _vp, ctypes.c_int, _vp]
@@ -135,6 +138,12 @@ def nvfp4_amax(x: torch.Tensor, amax_out: torch.Tensor) -> None:
     _check("nvfp4_amax", _lib.nvfp4_amax(_ptr(x), _in_dtype(x), M, K, _ptr(amax_out), _stream(x)))
 
 
+def nvfp4_amax_accumulate(x: torch.Tensor, running_amax: torch.Tensor) -> None:
+    M, K = x.shape
+    _check("nvfp4_amax_accumulate",
+           _lib.nvfp4_amax_accumulate(_ptr(x), _in_dtype(x), M, K, _ptr(running_amax), _stream(x)))
+
+
 def nvfp4_quantize(x: torch.Tensor, global_scale: float, codes: torch.Tensor, block_scales: torch.Tensor,
                    layout: int = SF_TCGEN05, amax_out: torch.Tensor | None = None) -> None:
     M, K = x.shape
@@ -188,6 +197,16 @@ def nvfp4_fused_proj(a_codes, a_scales, a_global_scale, w_codes, w_scales, seg_o
     _check("nvfp4_fused_proj",
            _lib.nvfp4_fused_proj(_ptr(a_codes), _ptr(a_scales), float(a_global_scale), _ptr(w_codes),
                                  _ptr(w_scales), offs, gs, n, M, K, _ptr(out), _out_dtype(out), _stream(out)))
+
+
+def nvfp4_harmonize_scales(scales: torch.Tensor, N: int, K: int, seg_offsets, seg_global_scales,
+                           common_global_scale: float, out: torch.Tensor, layout: int = SF_TCGEN05) -> None:
+    n = len(seg_global_scales)
+    offs = (_i64 * (n + 1))(*[int(v) for v in seg_offsets])
+    gs = (_f32 * n)(*[float(v) for v in seg_global_scales])
+    _check("nvfp4_harmonize_scales",
+           _lib.nvfp4_harmonize_scales(_ptr(scales), N, K, layout, offs, gs, n, float(common_global_scale),
+                                       _ptr(out), _stream(out)))
 
 
 def nvfp4_convert_e4m3(x: torch.Tensor, out: torch.Tensor) -> None:

@@ -1,6 +1,6 @@
 """Build libnvfp4.so (the C-ABI library) for sm_100a with nvcc, in-tree.
 
-    python -m nvfp4_w4a4_quantized_10_b200.build [--force] [--verbose]
+    python nvfp4_w4a4_quantized_10_b200/build.py [--force] [--verbose]
 
 Objects go to ``_build/`` next to this file; the shared library lands at
 ``nvfp4_w4a4_quantized_10_b200/libnvfp4.so``.  Only the CUDA runtime is
@@ -14,8 +14,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 SRC_DIR = os.path.join(HERE, "csrc")
 BUILD_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libnvfp4.so")
-SOURCES = ["runtime.cu", "quantize.cu", "gemm.cu"]
-HEADERS = ["ptx.cuh", "common.h", os.path.join("..", "..", "include", "nvfp4.h")]
+SOURCES = ["runtime.cu", "quantize.cu", "gemm.cu", "harmonize.cu"]
+HEADERS = ["ptx.cuh", "common.h", "block_quant.cuh", os.path.join("..", "..", "include", "nvfp4.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -114,24 +114,38 @@ __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ 
 }
 
 template <bool kF32>
+__device__ __forceinline__ float vec_absmax(const uint4& v, float m) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    if constexpr (kF32) {
+      m = fmaxf(m, fabsf(__uint_as_float(w[k])));
+    } else {
+      m = fmaxf(m, fabsf(__uint_as_float(w[k] << 16)));
+      m = fmaxf(m, fabsf(__uint_as_float(w[k] & 0xFFFF0000u)));
+    }
+  }
+  return m;
+}
+
+template <bool kF32>
 __global__ void __launch_bounds__(256) amax_kernel(const void* __restrict__ x, int64_t n_vec, float* amax_out) {
   // n_vec 16-byte vectors; any tail elements are handled by the host-chosen
   // element count being a multiple of the vector width (K*M*elt % 16 == 0).
+  // Launched as a programmatic dependent: the next kernel may start its
+  // prologue now; x is read only after the previous kernel has completed.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   float m = 0.0f;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_vec; i += stride) {
-    const uint4 v = __ldcs(reinterpret_cast<const uint4*>(x) + i);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      if constexpr (kF32) {
-        m = fmaxf(m, fabsf(__uint_as_float(w[k])));
-      } else {
-        m = fmaxf(m, fabsf(__uint_as_float(w[k] << 16)));
-        m = fmaxf(m, fabsf(__uint_as_float(w[k] & 0xFFFF0000u)));
-      }
-    }
+  const uint4* xv = reinterpret_cast<const uint4*>(x);
+  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (; i + stride < n_vec; i += 2 * stride) {  // two loads in flight per thread
+    const uint4 a = __ldcs(xv + i);
+    const uint4 b = __ldcs(xv + i + stride);
+    m = vec_absmax<kF32>(b, vec_absmax<kF32>(a, m));
   }
+  if (i < n_vec) m = vec_absmax<kF32>(__ldcs(xv + i), m);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
   __shared__ float wmax[8];
@@ -222,6 +236,21 @@ cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, float g, uint8_
                             scales, amax_out, kc);
 }
 
+cudaError_t launch_amax(const void* x, bool f32, int64_t n_vec, float* amax_out, cudaStream_t st,
+                        const DeviceInfo* d) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid_for(ceil_div(n_vec, 2), 256, d, 8));
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return f32 ? cudaLaunchKernelEx(&cfg, amax_kernel<true>, x, n_vec, amax_out)
+             : cudaLaunchKernelEx(&cfg, amax_kernel<false>, x, n_vec, amax_out);
+}
+
 }  // namespace
 }  // namespace nvfp4
 
@@ -248,11 +277,20 @@ nvfp4_status nvfp4_amax(const void* x, nvfp4_in_dtype dtype, int64_t M, int64_t 
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), st);
   if (e != cudaSuccess) return cuda_status(e);
-  const int64_t n_vec = M * K * elt / 16;
-  const int blocks = grid_for(n_vec, 256, d, 8);
-  if (dtype == NVFP4_IN_F32) amax_kernel<true><<<blocks, 256, 0, st>>>(x, n_vec, amax_out);
-  else amax_kernel<false><<<blocks, 256, 0, st>>>(x, n_vec, amax_out);
-  return cuda_status(cudaGetLastError());
+  return cuda_status(launch_amax(x, dtype == NVFP4_IN_F32, M * K * elt / 16, amax_out, st, d));
+}
+
+nvfp4_status nvfp4_amax_accumulate(const void* x, nvfp4_in_dtype dtype, int64_t M, int64_t K,
+                                   float* running_amax, nvfp4_stream_t stream) {
+  if (!x || !running_amax || M < 1 || K < 1) return NVFP4_ERR_INVALID_ARG;
+  if (dtype != NVFP4_IN_BF16 && dtype != NVFP4_IN_F32) return NVFP4_ERR_INVALID_ARG;
+  const int64_t elt = dtype == NVFP4_IN_F32 ? 4 : 2;
+  if ((M * K * elt) % 16 != 0) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(running_amax) & 3)) return NVFP4_ERR_ALIGNMENT;
+  const DeviceInfo* d = device_info();
+  if (!d) return NVFP4_ERR_CUDA;
+  return cuda_status(launch_amax(x, dtype == NVFP4_IN_F32, M * K * elt / 16, running_amax,
+                                 (cudaStream_t)stream, d));
 }
 
 nvfp4_status nvfp4_quantize(const void* x, nvfp4_in_dtype dtype, int64_t M, int64_t K, float global_scale,

@@ -107,6 +107,39 @@ def test_other_validation():
     assert L.nvfp4_test_wait_timeout(11_000_000_000, None) == nv.ERR_INVALID_ARG
 
 
+def harm(offs, gs, g=1.0, N=16, K=64, layout=1, sc=A16, out=A16, n_seg=None):
+    n = len(gs) if n_seg is None else n_seg
+    o = (ctypes.c_int64 * len(offs))(*offs)
+    s = (ctypes.c_float * max(1, len(gs)))(*gs)
+    return nv.lib().nvfp4_harmonize_scales(sc, N, K, layout, o, s, n, ctypes.c_float(g), out, None)
+
+
+def test_harmonize_and_calibration_validation():
+    assert harm([0, 8, 16], [1.0, 2.0], sc=None) == nv.ERR_INVALID_ARG
+    assert harm([0, 8, 16], [1.0, 2.0], out=None) == nv.ERR_INVALID_ARG
+    assert harm([0, 8, 16], [1.0, 2.0], N=0) == nv.ERR_INVALID_ARG
+    assert harm([0, 8, 16], [1.0, 2.0], K=24) == nv.ERR_INVALID_ARG
+    assert harm([0, 8, 16], [1.0, 2.0], layout=4) == nv.ERR_INVALID_ARG
+    assert harm([0, 8, 16], [1.0, 2.0], g=0.0) == nv.ERR_INVALID_ARG
+    assert harm([0, 8, 16], [1.0, 2.0], g=float("nan")) == nv.ERR_INVALID_ARG
+    assert harm([0, 8, 16], [1.0, -2.0]) == nv.ERR_INVALID_ARG             # bad segment scale
+    assert harm([0, 8, 8], [1.0, 2.0]) == nv.ERR_INVALID_ARG               # empty segment
+    assert harm([2, 8, 16], [1.0, 2.0]) == nv.ERR_INVALID_ARG              # does not start at 0
+    assert harm([0, 8, 17], [1.0, 2.0]) == nv.ERR_INVALID_ARG              # beyond N
+    assert harm([0, 8, 16], [1.0, 2.0], n_seg=0) == nv.ERR_INVALID_ARG
+    assert harm(list(range(17)), [1.0] * 17, N=32) == nv.ERR_INVALID_ARG   # too many
+    assert harm([0, 8, 16], [1.0, 2.0], sc=A1) == nv.ERR_ALIGNMENT
+    assert harm([0, 8, 16], [1.0, 2.0], out=A1) == nv.ERR_ALIGNMENT
+    L = nv.lib()
+    assert L.nvfp4_amax_accumulate(None, 0, 4, 64, A16, None) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_amax_accumulate(A16, 0, 4, 64, None, None) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_amax_accumulate(A16, 0, 0, 64, A16, None) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_amax_accumulate(A16, 0, 1, 4, A16, None) == nv.ERR_INVALID_ARG   # 8 bytes
+    assert L.nvfp4_amax_accumulate(A16, 5, 4, 64, A16, None) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_amax_accumulate(A1, 0, 4, 64, A16, None) == nv.ERR_ALIGNMENT
+    assert L.nvfp4_amax_accumulate(A16, 0, 4, 64, P(0x10002), None) == nv.ERR_ALIGNMENT
+
+
 def lin(x=A16, dt=0, M=8, K=64, ga=1.0, w=A16, sw=A16, gw=1.0, N=64, out=A16, od=0, ac=None, asc=None):
     return nv.lib().nvfp4_linear(x, dt, M, K, ctypes.c_float(ga), w, sw, ctypes.c_float(gw), N, out, od, ac, asc,
                                  None)
