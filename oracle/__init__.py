@@ -58,6 +58,13 @@ def lib():
         L.orc_saturation.argtypes = [f32p, i64, i64, ctypes.c_float, i64p]
         L.orc_harmonize_scales.argtypes = [u8p, i64, i64, i64p, f32p, ctypes.c_int,
                                            ctypes.c_float, u8p]
+        L.orc_e8m0_decode.restype = ctypes.c_double
+        L.orc_e8m0_decode.argtypes = [ctypes.c_uint8]
+        L.orc_mx_scale.restype = ctypes.c_uint8
+        L.orc_mx_scale.argtypes = [ctypes.c_float]
+        L.orc_mx_quantize.argtypes = [f32p, i64, i64, u8p, u8p]
+        L.orc_mx_dequantize.argtypes = [u8p, u8p, i64, i64, f64p]
+        L.orc_mx_gemm.argtypes = [u8p, u8p, u8p, u8p, i64, i64, i64, f64p]
         L.orc_set_threads.argtypes = [ctypes.c_int]
         L.orc_get_threads.restype = ctypes.c_int
         _lib = L
@@ -243,3 +250,54 @@ def harmonize_scales(scales, seg_offsets, seg_gs, g):
                                _p(gs, ctypes.c_float), len(gs), float(np.float32(g)),
                                _p(out, ctypes.c_uint8))
     return out
+
+
+# ---- MXFP4 (the contrast format) -------------------------------------------
+
+def e8m0_decode(b: int) -> float:
+    return float(lib().orc_e8m0_decode(b))
+
+
+def mx_scale(amax) -> int:
+    return int(lib().orc_mx_scale(float(np.float32(amax))))
+
+
+def mx_quantize(x):
+    """x: [M, K] float32 (K % 32 == 0). Returns (codes [M,K/2] u8, E8M0 scales [M,K/32] u8)."""
+    x = _c(x, np.float32)
+    M, K = x.shape
+    assert K % 32 == 0
+    codes = np.empty((M, K // 2), np.uint8)
+    scales = np.empty((M, K // 32), np.uint8)
+    lib().orc_mx_quantize(_p(x, ctypes.c_float), M, K, _p(codes, ctypes.c_uint8), _p(scales, ctypes.c_uint8))
+    return codes, scales
+
+
+def mx_dequantize(codes, scales):
+    codes, scales = _c(codes, np.uint8), _c(scales, np.uint8)
+    M, K = codes.shape[0], codes.shape[1] * 2
+    out = np.empty((M, K), np.float64)
+    lib().orc_mx_dequantize(_p(codes, ctypes.c_uint8), _p(scales, ctypes.c_uint8), M, K, _p(out, ctypes.c_double))
+    return out
+
+
+def mx_gemm(a_codes, a_scales, w_codes, w_scales):
+    a_codes, a_scales = _c(a_codes, np.uint8), _c(a_scales, np.uint8)
+    w_codes, w_scales = _c(w_codes, np.uint8), _c(w_scales, np.uint8)
+    M, K = a_codes.shape[0], a_codes.shape[1] * 2
+    N = w_codes.shape[0]
+    out = np.empty((M, N), np.float64)
+    lib().orc_mx_gemm(_p(a_codes, ctypes.c_uint8), _p(a_scales, ctypes.c_uint8), _p(w_codes, ctypes.c_uint8),
+                      _p(w_scales, ctypes.c_uint8), M, N, K, _p(out, ctypes.c_double))
+    return out
+
+
+def mx_scales_to_tc(rowmajor, K: int):
+    """MX scales [R, K/32] in the tensor-core chunk order.  The order depends
+    only on the scale matrix's shape (128 rows x 4 scales per 512-byte chunk),
+    so it is the NVFP4 order of a matrix with K/32 scales per row."""
+    return scales_to_tc(rowmajor, K // 2)
+
+
+def mx_scales_from_tc(tc, R: int, K: int):
+    return scales_from_tc(tc, R, K // 2)

@@ -449,3 +449,91 @@ void orc_harmonize_scales(const uint8_t* scales, int64_t R, int64_t K, const int
             }
     }
 }
+
+/* ------------------------------------------------------------------ */
+/* MXFP4, the contrast format (readings R16, R17)                      */
+/* ------------------------------------------------------------------ */
+
+/* The pages set NVFP4 against the MX format: blocks of 32 elements sharing
+ * one power-of-two scale, where NVFP4 uses 16 elements and an E4M3 scale
+ * [anthology record LIT-800, "Standing in the anthology"].  The conversion
+ * below is the published OCP Microscaling v1.0 rule for MXFP4, in the
+ * spec's order: per block of 32 along K,
+ *     E = floor(log2(max |x|)) - 2        (2: exponent of E2M1's largest
+ *                                           normal, 6 = 1.5 * 2^2)
+ * clamped to the E8M0 range [-127, 127]; the scale byte is E + 127 and
+ * every element is E2M1(x * 2^-E), nearest even, saturating at 6 (the
+ * quotient is exact: a power-of-two scaling of a float).  An all-zero
+ * block gets E = -127 (byte 0).  Value = e2m1(code) * 2^(byte - 127).
+ * There is no per-tensor scale.  Byte 255 (NaN) is never produced. */
+
+double orc_e8m0_decode(uint8_t b) {
+    return ldexp(1.0, (int)b - 127);
+}
+
+uint8_t orc_mx_scale(float amax) {
+    if (!(amax > 0.0f)) return 0;
+    int e2;
+    (void)frexp((double)amax, &e2);       /* amax = f * 2^e2, f in [0.5, 1) */
+    int E = (e2 - 1) - 2;                 /* floor(log2(amax)) - 2 */
+    if (E < -127) E = -127;
+    if (E > 127) E = 127;
+    return (uint8_t)(E + 127);
+}
+
+/* x: [M, K] FP32, K a multiple of 32.  codes: [M, K/2] (element 2j in the
+ * low nibble of byte j); scales: [M, K/32] E8M0 bytes, row-major. */
+void orc_mx_quantize(const float* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* scales) {
+    const int64_t nb = K / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t b = 0; b < nb; ++b) {
+            const float* xb = x + m * K + b * 32;
+            float amax = 0.0f;
+            for (int i = 0; i < 32; ++i) {
+                float a = fabsf(xb[i]);
+                if (a > amax) amax = a;
+            }
+            uint8_t s = orc_mx_scale(amax);
+            scales[m * nb + b] = s;
+            int E = (int)s - 127;
+            uint8_t c[32];
+            for (int i = 0; i < 32; ++i) {
+                float y = (float)ldexp((double)xb[i], -E);
+                c[i] = orc_e2m1_encode(y);
+            }
+            uint8_t* cb = codes + m * (K / 2) + b * 16;
+            for (int j = 0; j < 16; ++j)
+                cb[j] = (uint8_t)(c[2 * j] | (c[2 * j + 1] << 4));
+        }
+    }
+}
+
+void orc_mx_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t M, int64_t K, double* out) {
+    const int64_t nb = K / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t k = 0; k < K; ++k) {
+            uint8_t byte = codes[m * (K / 2) + k / 2];
+            uint8_t code = (k & 1) ? (byte >> 4) : (byte & 0xF);
+            out[m * K + k] = orc_e2m1_decode(code) * orc_e8m0_decode(scales[m * nb + k / 32]);
+        }
+}
+
+/* out[m,n] = sum_k deqA[m,k] * deqW[n,k] in FP64, MXFP4 operands. */
+void orc_mx_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* w_codes,
+                 const uint8_t* w_scales, int64_t M, int64_t N, int64_t K, double* out) {
+    double* da = (double*)malloc(sizeof(double) * (size_t)(M * K));
+    double* dw = (double*)malloc(sizeof(double) * (size_t)(N * K));
+    orc_mx_dequantize(a_codes, a_scales, M, K, da);
+    orc_mx_dequantize(w_codes, w_scales, N, K, dw);
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t m = 0; m < M; ++m) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) acc += da[m * K + k] * dw[n * K + k];
+            out[m * N + n] = acc;
+        }
+    free(da);
+    free(dw);
+}
