@@ -669,13 +669,114 @@ def measure_harmonize(torch, nv, synth, dev, rank, l2, args, stream, peaks):
     return res
 
 
+def measure_mx(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind):
+    """MXFP4, the contrast format: its quantizer (X[4096,5120] bf16), its
+    kind::mxf4 GEMM on the prefill and decode shapes (weights rotated through
+    copies larger than L2), and the GEMM error of NVFP4 and MXFP4 against the
+    FP64 product of the unquantized operands, on the prefill activation
+    recipe (outlier channels at 63x RMS)."""
+    hbm_peak = float(peaks["hbm_gbs"])
+    tc_peak = float(peaks["bf16_tflops"]) * FP4_OVER_BF16
+    res = {}
+    kk = max(3, min(args.steps, 50))
+    # quantizer
+    M, K = 4096, 5120
+    xs = [synth.activation(synth.PREFILL, device=dev, M=M, seed=synth.PREFILL.seed + 1000 * rank)]
+    xs += [xs[0].clone() for _ in range(3)]
+    qc, qs = nv.alloc_mx_quantized(M, K, dev)
+
+    def q(i):
+        nv.nvfp4_mx_quantize(xs[i % 4], qc, qs)
+
+    with torch.cuda.stream(stream):
+        ms_q, g1 = time_graph(torch, q, kk, 3, stream)
+    del g1
+    qb = M * K * 2 + M * K // 2 + M * K // 32
+    res["quantize_4096x5120"] = {"us": ms_q * 1e3, "GB/s": qb / (ms_q * 1e-3) / 1e9,
+                                 "frac_hbm": qb / (ms_q * 1e-3) / 1e9 / hbm_peak}
+    # prefill-shape GEMM
+    w = synth.PREFILL
+    pm = args.prefill_m or w.M
+    x = synth.activation(w, device=dev, M=pm, seed=w.seed + 1000 * rank)
+    wt = synth.weight(w, device=dev)
+    ac, as_ = nv.alloc_mx_quantized(pm, w.K, dev)
+    wc, ws = nv.alloc_mx_quantized(w.N, w.K, dev)
+    nv.nvfp4_mx_quantize(x, ac, as_)
+    nv.nvfp4_mx_quantize(wt, wc, ws)
+    del x, wt
+    out = torch.empty(pm, w.N, dtype=torch.bfloat16, device=dev)
+
+    def gp(i):
+        nv.nvfp4_mx_gemm(ac, as_, wc, ws, pm, w.N, w.K, out)
+
+    with torch.cuda.stream(stream):
+        ms_p, g2 = time_graph(torch, gp, max(3, min(args.steps, 10)), 3, stream)
+    del g2
+    fl = 2.0 * pm * w.N * w.K
+    res["gemm_prefill"] = {"shape": [pm, w.N, w.K], "ms": ms_p, "TFLOP/s": fl / (ms_p * 1e-3) / 1e12,
+                           "frac_fp4_peak": fl / (ms_p * 1e-3) / 1e12 / tc_peak, "peak": peak_kind}
+    del ac, as_, wc, ws, out
+    # decode-shape GEMM
+    d = synth.DECODE
+    x = synth.activation(d, device=dev, seed=d.seed + 1000 * rank)
+    wt = synth.weight(d, device=dev)
+    ac, as_ = nv.alloc_mx_quantized(d.M, d.K, dev)
+    nv.nvfp4_mx_quantize(x, ac, as_)
+    wc, ws = nv.alloc_mx_quantized(d.N, d.K, dev)
+    nv.nvfp4_mx_quantize(wt, wc, ws)
+    per = wc.numel() + ws.numel()
+    n_copies = max(2, math.ceil(3 * l2 / per))
+    copies = [(wc, ws)] + [(wc.clone(), ws.clone()) for _ in range(n_copies - 1)]
+    out = torch.empty(d.M, d.N, dtype=torch.bfloat16, device=dev)
+
+    def gd(i):
+        c, s_ = copies[i % n_copies]
+        nv.nvfp4_mx_gemm(ac, as_, c, s_, d.M, d.N, d.K, out)
+
+    with torch.cuda.stream(stream):
+        ms_d, g3 = time_graph(torch, gd, kk, 3, stream)
+    del g3
+    db = ac.numel() + as_.numel() + per + d.M * d.N * 2
+    res["gemm_decode"] = {"shape": [d.M, d.N, d.K], "us": ms_d * 1e3, "GB/s": db / (ms_d * 1e-3) / 1e9,
+                          "frac_hbm": db / (ms_d * 1e-3) / 1e9 / hbm_peak}
+    del copies, wc, ws, ac, as_, x, wt
+    # accuracy against the FP64 product of the unquantized operands
+    M, N, K = 4096, 4096, w.K
+    x = synth.activation(w, device=dev, M=M)
+    wt = synth.weight(w, device=dev, N=N)
+    ref = x.double() @ wt.double().T
+    am = torch.empty(1, dtype=torch.float32, device=dev)
+    nv.nvfp4_amax(x, am)
+    ga = 2688.0 / am.item()
+    nv.nvfp4_amax(wt, am)
+    gw = 2688.0 / am.item()
+    a_c, a_s = nv.alloc_quantized(M, K, dev)
+    w_c, w_s = nv.alloc_quantized(N, K, dev)
+    nv.nvfp4_quantize(x, ga, a_c, a_s)
+    nv.nvfp4_quantize(wt, gw, w_c, w_s)
+    o_nv = torch.empty(M, N, dtype=torch.float32, device=dev)
+    nv.nvfp4_gemm(a_c, a_s, ga, w_c, w_s, gw, M, N, K, o_nv)
+    ma, mas = nv.alloc_mx_quantized(M, K, dev)
+    mw, mws = nv.alloc_mx_quantized(N, K, dev)
+    nv.nvfp4_mx_quantize(x, ma, mas)
+    nv.nvfp4_mx_quantize(wt, mw, mws)
+    o_mx = torch.empty_like(o_nv)
+    nv.nvfp4_mx_gemm(ma, mas, mw, mws, M, N, K, o_mx)
+    torch.cuda.synchronize()
+    res["gemm_rel_fro_vs_unquantized"] = {
+        "workload": f"X[{M},{K}] prefill recipe x W[{N},{K}] N(0,0.02)",
+        "nvfp4": float((o_nv.double() - ref).norm() / ref.norm()),
+        "mxfp4": float((o_mx.double() - ref).norm() / ref.norm())}
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--only", default="all", choices=["all", "decode", "prefill", "fused", "quant", "calib", "harmonize"])
+    ap.add_argument("--only", default="all", choices=["all", "decode", "prefill", "fused", "quant", "calib", "harmonize", "mx"])
     ap.add_argument("--prefill-m", type=int, default=0, help="override M of the prefill workload")
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed decode steps first")
     ap.add_argument("--no-extra", action="store_true")
@@ -729,6 +830,8 @@ def main():
             res = measure_calibration(torch, nv, synth, dev, args, stream, peaks)
         elif args.only == "harmonize":
             res = measure_harmonize(torch, nv, synth, dev, rank, l2, args, stream, peaks)
+        elif args.only == "mx":
+            res = measure_mx(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind)
         else:
             res = measure_quant_sweep(torch, nv, synth, dev, args, stream, peaks)
         sampler.stop()
@@ -745,6 +848,7 @@ def main():
             "quantize_sweep": measure_quant_sweep(torch, nv, synth, dev, args, stream, peaks),
             "static_calibration": measure_calibration(torch, nv, synth, dev, args, stream, peaks),
             "harmonize": measure_harmonize(torch, nv, synth, dev, rank, l2, args, stream, peaks),
+            "mxfp4": measure_mx(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind),
         }
     sampler.stop()
     if clk is not None:

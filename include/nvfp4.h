@@ -279,6 +279,37 @@ NVFP4_API nvfp4_status nvfp4_harmonize_scales(const uint8_t* scales, int64_t N, 
                                     const int64_t* seg_offsets, const float* seg_global_scales, int n_seg,
                                     float common_global_scale, uint8_t* out, nvfp4_stream_t stream);
 
+/* MXFP4, the contrast format: 32-element blocks sharing one power-of-two
+ * (E8M0) scale and no per-tensor scale, where NVFP4 uses 16-element blocks
+ * with an E4M3 scale [anthology record LIT-800, "Standing in the anthology":
+ * NVFP4's finer blocks keep outliers local].  Conversion (the OCP
+ * Microscaling v1.0 rule for MXFP4): per block of 32 along K,
+ *   E = floor(log2(max |x|)) - 2, clamped to [-127, 127];  scale byte E + 127;
+ *   code_i = E2M1(x_i * 2^-E) (nearest even, saturating at 6); an all-zero
+ *   block gets byte 0.  Value = e2m1(code) * 2^(byte - 127).
+ *   x       device [M, K] bf16/f32 row-major, 16-byte aligned; K % 32 == 0;
+ *           finite (NaN or infinite inputs give unspecified bytes)
+ *   codes   device [M, K/2] bytes (element 2j in the low nibble of byte j)
+ *   scales  device, nvfp4_scale_bytes(M, K/2, layout) bytes, 16-byte aligned:
+ *           row-major [M, K/32], or the TCGEN05 chunk order with 4 scales
+ *           (128 K-elements) per row of a 512-byte chunk, padding written 0.
+ * Errors: INVALID_ARG (null, M < 1, K < 32 or K % 32, bad dtype or layout),
+ * UNSUPPORTED (M*K/16 >= 2^31), ALIGNMENT, CUDA. */
+NVFP4_API nvfp4_status nvfp4_mx_quantize(const void* x, nvfp4_in_dtype dtype, int64_t M, int64_t K, uint8_t* codes,
+                               uint8_t* scales, nvfp4_sf_layout layout, nvfp4_stream_t stream);
+
+/* MXFP4 x MXFP4 GEMM on the tensor cores (tcgen05.mma kind::mxf4, two E8M0
+ * scales per row per K=64 step):  out[m,n] = sum_k deqA[m,k] * deqW[n,k],
+ * accumulated in FP32, then bf16 (nearest even) or f32.  The same kernel,
+ * tiling, split-K decode path and workspace as nvfp4_gemm; the scales are
+ * those of nvfp4_mx_quantize in the TCGEN05 layout.
+ *   a_codes/a_scales [M, K/2] and nvfp4_scale_bytes(M, K/2, TCGEN05) bytes;
+ *   w_codes/w_scales [N, K/2] and nvfp4_scale_bytes(N, K/2, TCGEN05) bytes;
+ *   other arguments, limits and errors as nvfp4_gemm. */
+NVFP4_API nvfp4_status nvfp4_mx_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* w_codes,
+                           const uint8_t* w_scales, int64_t M, int64_t N, int64_t K, void* out,
+                           nvfp4_out_dtype out_dtype, nvfp4_stream_t stream);
+
 /* Element conversions exactly as the quantizer performs them, exposed so the
  * encoders can be checked exhaustively.
  *   nvfp4_convert_e4m3: out[i] = E4M3(in[i]) (nearest-even, saturating).

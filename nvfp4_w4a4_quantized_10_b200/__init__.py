@@ -45,6 +45,8 @@ _lib.nvfp4_amax.argtypes = [_vp, ctypes.c_int, _i64, _i64, _vp, _vp]
 _lib.nvfp4_amax_accumulate.argtypes = [_vp, ctypes.c_int, _i64, _i64, _vp, _vp]
 _lib.nvfp4_harmonize_scales.argtypes = [_vp, _i64, _i64, ctypes.c_int, ctypes.POINTER(_i64), ctypes.POINTER(_f32),
                                         ctypes.c_int, _f32, _vp, _vp]
+_lib.nvfp4_mx_quantize.argtypes = [_vp, ctypes.c_int, _i64, _i64, _vp, _vp, ctypes.c_int, _vp]
+_lib.nvfp4_mx_gemm.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_int, _vp]
 _lib.nvfp4_quantize.argtypes = [_vp, ctypes.c_int, _i64, _i64, _f32, _vp, _vp, ctypes.c_int, _vp, _vp]
 _lib.nvfp4_swizzle_scales.argtypes = [_vp, _i64, _i64, _vp, _vp]
 _lib.nvfp4_gemm.argtypes = [_vp, _vp, _f32, _vp, _vp, _f32, _i64, _i64, _i64, _vp, ctypes.c_int, _vp]
@@ -207,6 +209,24 @@ def nvfp4_harmonize_scales(scales: torch.Tensor, N: int, K: int, seg_offsets, se
     _check("nvfp4_harmonize_scales",
            _lib.nvfp4_harmonize_scales(_ptr(scales), N, K, layout, offs, gs, n, float(common_global_scale),
                                        _ptr(out), _stream(out)))
+
+
+def nvfp4_mx_quantize(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, layout: int = SF_TCGEN05) -> None:
+    M, K = x.shape
+    _check("nvfp4_mx_quantize", _lib.nvfp4_mx_quantize(_ptr(x), _in_dtype(x), M, K, _ptr(codes), _ptr(scales),
+                                                       layout, _stream(x)))
+
+
+def alloc_mx_quantized(rows: int, K: int, device, layout: int = SF_TCGEN05):
+    """Empty MXFP4 code and scale buffers for a [rows, K] operand."""
+    codes = torch.empty(rows, K // 2, dtype=torch.uint8, device=device)
+    scales = torch.empty(nvfp4_scale_bytes(rows, K // 2, layout), dtype=torch.uint8, device=device)
+    return codes, scales
+
+
+def nvfp4_mx_gemm(a_codes, a_scales, w_codes, w_scales, M, N, K, out: torch.Tensor) -> None:
+    _check("nvfp4_mx_gemm", _lib.nvfp4_mx_gemm(_ptr(a_codes), _ptr(a_scales), _ptr(w_codes), _ptr(w_scales), M, N,
+                                               K, _ptr(out), _out_dtype(out), _stream(out)))
 
 
 def nvfp4_convert_e4m3(x: torch.Tensor, out: torch.Tensor) -> None:

@@ -71,7 +71,8 @@ struct alignas(64) GemmParams {
   int64_t M, N;          // output [M, N]
   int rows_p, rows_q;    // rows of the P and Q operands
   int rb_q;              // 128-row scale blocks allocated for Q
-  int kc;                // ceil(K / 64): scale chunks per row block
+  int kc;                // scale chunks per row block: ceil(K / 64), MXFP4 ceil(K / 128)
+  int kmma;              // ceil(K / 64): MMAs per row of tiles
   int kt;                // ceil(K / (64 * kKB)): pipeline steps per tile
   int tiles_p, tiles_q;
   int tma_store;         // 1: output through shared memory and TMA stores
@@ -90,7 +91,9 @@ struct alignas(64) GemmParams {
 // in global memory; 1 / 2 = swapped tiles whose activation X (bf16 / f32) the
 // kernel quantizes itself into shared memory, all of the CTA's K-steps at
 // once, before the first MMA.
-template <int BN, bool SWAP, int QX = 0>
+// MX: MXFP4 operands (32-element blocks, E8M0 scales, kind::mxf4 with two
+// scales per MMA) instead of NVFP4 (16-element blocks, E4M3 scales).
+template <int BN, bool SWAP, int QX = 0, bool MX = false>
 struct Cfg {
   static constexpr bool kQx = QX != 0;
   // K per pipeline step: kKB blocks of 64 (one MMA each), 256 deep, as
@@ -105,8 +108,11 @@ struct Cfg {
   static constexpr int kSfbBlocks = (BN + 127) / 128;                // 128-row scale blocks of Q
   static constexpr int kABytes = kBM * kRowBytes;
   static constexpr int kBBytes = kQx ? 0 : BN * kRowBytes;           // Q codes per stage
-  static constexpr int kSfaBytes = kKB * kSfChunk;
-  static constexpr int kSfbBytes = kQx ? 0 : kSfbBlocks * kKB * kSfChunk;
+  // scale chunks (128 rows x 4 scales, 512 bytes) per step: a chunk covers 64
+  // K-elements of 16-element blocks (one MMA), or 128 of 32-element blocks
+  static constexpr int kChunks = MX ? kKB / 2 : kKB;
+  static constexpr int kSfaBytes = kChunks * kSfChunk;
+  static constexpr int kSfbBytes = kQx ? 0 : kSfbBlocks * kChunks * kSfChunk;
   static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
   static constexpr int kOutBytes = SWAP ? 0 : 2 * kStageOutBytes;    // double-buffered output sub-tiles
   // in-kernel activation: codes (BN rows x 128 B, 128B swizzle) and one
@@ -150,8 +156,8 @@ struct Cfg {
   // pipeline stage.
   static constexpr int kAccCols = BN < 32 ? 32 : BN;
   static constexpr bool kOverlapAcc = !SWAP && BN == 256;
-  static constexpr int kSfaCols = 4 * kKB;                           // kKB MMAs x 4 columns
-  static constexpr int kSfbCols = kSfbBlocks * 4 * kKB;
+  static constexpr int kSfaCols = 4 * kChunks;                       // 4 columns per chunk
+  static constexpr int kSfbCols = kSfbBlocks * 4 * kChunks;
   static constexpr int kSfStageCols = kSfaCols + kSfbCols;
   // four regions (192 columns) let the copy warps run up to three steps
   // ahead; the accumulators then share 192 columns (3 slots drained first)
@@ -165,6 +171,7 @@ struct Cfg {
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(BN % 16 == 0 && BN <= 256, "MMA N");
   static_assert(!kQx || (SWAP && BN <= 32), "in-kernel activation: swapped tiles, M <= 32");
+  static_assert(!(kQx && MX), "in-kernel activation: NVFP4 only");
   static_assert(kOffAct % 1024 == 0 && kActCodeBytes % 1024 == 0, "activation tiles on swizzle atoms");
 };
 
@@ -272,10 +279,10 @@ __device__ __forceinline__ uint64_t ld_word(const uint64_t* p) {
 // stored with the 128B swizzle the output tensor map uses.
 __device__ __forceinline__ uint32_t swz128(uint32_t r, uint32_t c) { return r * 128 + ((c ^ (r & 7)) << 4); }
 
-template <int BN, bool SWAP, bool OUT_F32, int QX = 0>
-__global__ void __launch_bounds__(Cfg<BN, SWAP, QX>::kThreads, 1)
+template <int BN, bool SWAP, bool OUT_F32, int QX = 0, bool MX = false>
+__global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ GemmParams p) {
-  using C = Cfg<BN, SWAP, QX>;
+  using C = Cfg<BN, SWAP, QX, MX>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -355,24 +362,24 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX>::kThreads, 1)
       };
       auto load_p = [&](int stage, int p0, int k) {
         const uint32_t fb = bar_full + 8 * stage;
-        const uint32_t sf_bytes = (uint32_t)min(C::kKB, kc - C::kKB * k) * kSfChunk;
+        const uint32_t sf_bytes = (uint32_t)min(C::kChunks, kc - C::kChunks * k) * kSfChunk;
         tma_load_2d(sbase + C::kOffA + stage * C::kABytes, &p.tmap_p, k * C::kRowBytes, p0, fb);
         bulk_load(sbase + C::kOffSfa + stage * C::kSfaBytes,
-                  p.sf_p + ((size_t)(p0 >> 7) * kc + C::kKB * k) * kSfChunk, sf_bytes, fb);
+                  p.sf_p + ((size_t)(p0 >> 7) * kc + C::kChunks * k) * kSfChunk, sf_bytes, fb);
       };
       auto load_q = [&](int stage, int q0, int k) {
         const uint32_t fb = bar_full + 8 * stage;
-        const uint32_t sf_bytes = (uint32_t)min(C::kKB, kc - C::kKB * k) * kSfChunk;
+        const uint32_t sf_bytes = (uint32_t)min(C::kChunks, kc - C::kChunks * k) * kSfChunk;
         const int nsfb = nsfb_of(q0);
         tma_load_2d(sbase + C::kOffB + stage * C::kBBytes, &p.tmap_q, k * C::kRowBytes, q0, fb);
 #pragma unroll
         for (int rb = 0; rb < C::kSfbBlocks; ++rb)
           if (rb < nsfb)
-            bulk_load(sbase + C::kOffSfb + stage * C::kSfbBytes + rb * C::kKB * kSfChunk,
-                      p.sf_q + ((size_t)((q0 >> 7) + rb) * kc + C::kKB * k) * kSfChunk, sf_bytes, fb);
+            bulk_load(sbase + C::kOffSfb + stage * C::kSfbBytes + rb * C::kChunks * kSfChunk,
+                      p.sf_q + ((size_t)((q0 >> 7) + rb) * kc + C::kChunks * k) * kSfChunk, sf_bytes, fb);
       };
       auto expect = [&](int stage, int q0, int k) {
-        const uint32_t sf_bytes = (uint32_t)min(C::kKB, kc - C::kKB * k) * kSfChunk;
+        const uint32_t sf_bytes = (uint32_t)min(C::kChunks, kc - C::kChunks * k) * kSfChunk;
         mbar_arrive_expect_tx(bar_full + 8 * stage,
                               C::kABytes + C::kBBytes + sf_bytes * (1 + (C::kQx ? 0 : nsfb_of(q0))));
       };
@@ -389,10 +396,10 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX>::kThreads, 1)
           else load_q(j, q0, k);
           issued_mask |= 1u << j;
         } else {
-          const uint32_t sf_bytes = (uint32_t)min(C::kKB, kc - C::kKB * k) * kSfChunk;
+          const uint32_t sf_bytes = (uint32_t)min(C::kChunks, kc - C::kChunks * k) * kSfChunk;
           if (SWAP) {
             tma_prefetch_l2_2d(&p.tmap_p, k * C::kRowBytes, p0);
-            bulk_prefetch_l2(p.sf_p + ((size_t)(p0 >> 7) * kc + C::kKB * k) * kSfChunk, sf_bytes);
+            bulk_prefetch_l2(p.sf_p + ((size_t)(p0 >> 7) * kc + C::kChunks * k) * kSfChunk, sf_bytes);
           } else {
             tma_prefetch_l2_2d(&p.tmap_q, k * C::kRowBytes, q0);
           }
@@ -440,7 +447,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX>::kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     // The whole warp follows the pipeline; lane 0 issues every MMA.  The copy
     // warps waited for each stage's data and moved its scales into TMEM.
-    constexpr uint32_t idesc = idesc_nvf4(kBM, BN);
+    constexpr uint32_t idesc = MX ? idesc_mxf4(kBM, BN) : idesc_nvf4(kBM, BN);
     // Descriptors of stage 0, k-block 0; later stages and k-blocks only move
     // the 14-bit start-address field (address >> 4), which never carries.
     const uint64_t a_desc0 = smem_desc(sbase + C::kOffA, 16, C::kSbo, C::kSwizzleLayout);
@@ -471,16 +478,22 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX>::kThreads, 1)
           const uint64_t ad = a_desc0 + (uint64_t)((stage * C::kABytes) >> 4);
           const uint64_t bd = b_desc0 + (uint64_t)(((C::kQx ? lstep * C::kActCodeBytes : stage * C::kBBytes)) >> 4);
           const uint32_t acc_in = k != kb0 ? 1u : 0u;
-          const int nkb = min(C::kKB, kc - C::kKB * k);
+          // MMA kb reads chunk kb (NVFP4, 4 scales each) or half of chunk
+          // kb / 2 (MXFP4: scale bytes 0-1 or 2-3 of each TMEM column,
+          // selected by the descriptor's scale-factor ids)
+          const int nkb = min(C::kKB, p.kmma - C::kKB * k);
+          auto mma = [&](int kb) {
+            const int c = MX ? kb >> 1 : kb;
+            const uint32_t id = MX ? (uint32_t)(kb & 1) * 2u : 0u;
+            tc_mma_block_scaled<MX>(acc, ad + (uint64_t)(kb * 2), bd + (uint64_t)(kb * 2),
+                                    idesc | (id << 29) | (id << 4), sfa_t + c * 4, sfb_t + c * 4 * C::kSfbBlocks,
+                                    (acc_in | kb) != 0 ? 1u : 0u);
+          };
           if (nkb == C::kKB) {
 #pragma unroll
-            for (int kb = 0; kb < C::kKB; ++kb)
-              tc_mma_nvf4(acc, ad + (uint64_t)(kb * 2), bd + (uint64_t)(kb * 2), idesc, sfa_t + kb * 4,
-                          sfb_t + kb * 4 * C::kSfbBlocks, (acc_in | kb) != 0 ? 1u : 0u);
+            for (int kb = 0; kb < C::kKB; ++kb) mma(kb);
           } else {
-            for (int kb = 0; kb < nkb; ++kb)
-              tc_mma_nvf4(acc, ad + (uint64_t)(kb * 2), bd + (uint64_t)(kb * 2), idesc, sfa_t + kb * 4,
-                          sfb_t + kb * 4 * C::kSfbBlocks, (acc_in | kb) != 0 ? 1u : 0u);
+            for (int kb = 0; kb < nkb; ++kb) mma(kb);
           }
           tc_commit(bar_empty + 8 * stage);
         }
@@ -920,22 +933,22 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX>::kThreads, 1)
             tc_fence_after();
           }
           const uint32_t sfa_t = sf_t0 + region * C::kSfStageCols;
-          const int nkb = min(C::kKB, kc - C::kKB * k);
+          const int nch = min(C::kChunks, kc - C::kChunks * k);
           if (copy_p) {
             const uint64_t d = desc0 + (uint64_t)((stage * C::kSfaBytes) >> 4);
-            if (nkb == C::kKB) {
+            if (nch == C::kChunks) {
 #pragma unroll
-              for (int kb = 0; kb < C::kKB; ++kb)
-                tc_cp_32x128b_warpx4(sfa_t + kb * 4, d + (uint64_t)(kb * (kSfChunk >> 4)));
+              for (int c = 0; c < C::kChunks; ++c)
+                tc_cp_32x128b_warpx4(sfa_t + c * 4, d + (uint64_t)(c * (kSfChunk >> 4)));
             } else {
-              for (int kb = 0; kb < nkb; ++kb) tc_cp_32x128b_warpx4(sfa_t + kb * 4, d + (uint64_t)(kb * (kSfChunk >> 4)));
+              for (int c = 0; c < nch; ++c) tc_cp_32x128b_warpx4(sfa_t + c * 4, d + (uint64_t)(c * (kSfChunk >> 4)));
             }
           } else {
             const uint64_t d = desc0 + (uint64_t)((C::kQx ? step * C::kActSfBytes : stage * C::kSfbBytes) >> 4);
             const uint32_t sfb_t = sfa_t + C::kSfaCols;
-            for (int kb = 0; kb < nkb; ++kb)
-              tc_cp_32x128b_warpx4(sfb_t + kb * 4 * C::kSfbBlocks + rbq * 4,
-                                   d + (uint64_t)((rbq * C::kKB + kb) * (kSfChunk >> 4)));
+            for (int c = 0; c < nch; ++c)
+              tc_cp_32x128b_warpx4(sfb_t + c * 4 * C::kSfbBlocks + rbq * 4,
+                                   d + (uint64_t)((rbq * C::kChunks + c) * (kSfChunk >> 4)));
           }
           tc_commit(bar_sf + 8 * stage);
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
@@ -1058,10 +1071,10 @@ cudaError_t get_workspace(const DeviceInfo* d, cudaStream_t st, Workspace* out) 
   return cudaSuccess;
 }
 
-template <int BN, bool SWAP, bool OUT_F32, int QX = 0>
+template <int BN, bool SWAP, bool OUT_F32, int QX = 0, bool MX = false>
 cudaError_t launch(const GemmParams& p, const DeviceInfo* d, cudaStream_t st) {
-  using Cf = Cfg<BN, SWAP, QX>;
-  auto kern = nvfp4_gemm_kernel<BN, SWAP, OUT_F32, QX>;
+  using Cf = Cfg<BN, SWAP, QX, MX>;
+  auto kern = nvfp4_gemm_kernel<BN, SWAP, OUT_F32, QX, MX>;
   static std::once_flag once[64];
   static cudaError_t attr_err[64];
   std::call_once(once[d->device], [&] {
@@ -1094,9 +1107,22 @@ cudaError_t launch(const GemmParams& p, const DeviceInfo* d, cudaStream_t st) {
 
 float alpha_of(float ga, float gw) { return (float)(1.0 / ((double)ga * (double)gw)); }
 
+template <bool MX>
+cudaError_t launch_shape(const GemmParams& p, const DeviceInfo* d, cudaStream_t st, bool swap, int bn, bool f32) {
+  if (!swap) return f32 ? launch<256, false, true, 0, MX>(p, d, st) : launch<256, false, false, 0, MX>(p, d, st);
+  if (bn == 16) return f32 ? launch<16, true, true, 0, MX>(p, d, st) : launch<16, true, false, 0, MX>(p, d, st);
+  if (bn == 32) return f32 ? launch<32, true, true, 0, MX>(p, d, st) : launch<32, true, false, 0, MX>(p, d, st);
+  if (bn == 64) return f32 ? launch<64, true, true, 0, MX>(p, d, st) : launch<64, true, false, 0, MX>(p, d, st);
+  return f32 ? launch<128, true, true, 0, MX>(p, d, st) : launch<128, true, false, 0, MX>(p, d, st);
+}
+
+// mx: MXFP4 operands (E8M0 scales of 32-element blocks, in the same chunk
+// order with 4 scales = 128 K-elements per chunk); the caller passes unit
+// global scales, so alpha = 1.
 nvfp4_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float ga, const uint8_t* w_codes,
                       const uint8_t* w_scales, const int64_t* seg_offsets, const float* seg_gs, int n_seg,
-                      int64_t M, int64_t N, int64_t K, void* out, nvfp4_out_dtype out_dtype, cudaStream_t st) {
+                      int64_t M, int64_t N, int64_t K, void* out, nvfp4_out_dtype out_dtype, cudaStream_t st,
+                      bool mx = false) {
   if (!a_codes || !a_scales || !w_codes || !w_scales || !out) return NVFP4_ERR_INVALID_ARG;
   if (M < 1 || N < 1 || K < 32 || K % 32 != 0) return NVFP4_ERR_INVALID_ARG;
   if (M > (1ll << 31) - 256 || N > (1ll << 31) - 256 || K > (1ll << 31)) return NVFP4_ERR_UNSUPPORTED;
@@ -1140,7 +1166,7 @@ nvfp4_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float ga,
   const bool f32 = out_dtype == NVFP4_OUT_F32;
   p.tma_store = (!swap && (N * (f32 ? 4 : 2)) % 16 == 0) ? 1 : 0;
   p.w_static = is_static(w_codes, (size_t)N * (size_t)(K / 2)) &&
-                       is_static(w_scales, nvfp4_scale_bytes(N, K, NVFP4_SF_TCGEN05))
+                       is_static(w_scales, nvfp4_scale_bytes(N, mx ? K / 2 : K, NVFP4_SF_TCGEN05))
                    ? 1 : 0;
   if (p.tma_store && !make_out_map(&p.tmap_out, out, M, N, f32)) return NVFP4_ERR_CUDA;
   p.err = d->err_word;
@@ -1148,7 +1174,8 @@ nvfp4_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float ga,
   p.M = M;
   p.N = N;
   p.rb_q = (int)ceil_div(p.rows_q, 128);
-  p.kc = (int)ceil_div(K, 64);
+  p.kc = (int)ceil_div(K, mx ? 128 : 64);
+  p.kmma = (int)ceil_div(K, 64);
   p.kt = (int)ceil_div(K, 64 * kkb);
   p.tiles_p = (int)ceil_div(p.rows_p, kBM);
   p.tiles_q = (int)ceil_div(p.rows_q, bn);
@@ -1157,13 +1184,7 @@ nvfp4_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float ga,
     p.seg_end[i] = (int)seg_offsets[i + 1];
     p.seg_alpha[i] = alpha_of(ga, seg_gs[i]);
   }
-  cudaError_t e;
-  if (!swap) e = f32 ? launch<256, false, true>(p, d, st) : launch<256, false, false>(p, d, st);
-  else if (bn == 16) e = f32 ? launch<16, true, true>(p, d, st) : launch<16, true, false>(p, d, st);
-  else if (bn == 32) e = f32 ? launch<32, true, true>(p, d, st) : launch<32, true, false>(p, d, st);
-  else if (bn == 64) e = f32 ? launch<64, true, true>(p, d, st) : launch<64, true, false>(p, d, st);
-  else e = f32 ? launch<128, true, true>(p, d, st) : launch<128, true, false>(p, d, st);
-  return cuda_status(e);
+  return cuda_status(mx ? launch_shape<true>(p, d, st, swap, bn, f32) : launch_shape<false>(p, d, st, swap, bn, f32));
 }
 
 // ---------------------------------------------------------------------------
@@ -1262,6 +1283,7 @@ nvfp4_status run_linear(const void* x, nvfp4_in_dtype x_dtype, int64_t M, int64_
   p.N = N;
   p.rb_q = 1;
   p.kc = (int)ceil_div(K, 64);
+  p.kmma = (int)ceil_div(K, 64);
   p.kt = (int)ceil_div(K, 64 * kkb);
   p.tiles_p = (int)ceil_div(p.rows_p, kBM);
   p.tiles_q = 1;
@@ -1344,6 +1366,7 @@ nvfp4_status run_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_scales, f
   p.N = N;
   p.rb_q = (int)ceil_div(p.rows_q, 128);
   p.kc = (int)ceil_div(K, 64);
+  p.kmma = (int)ceil_div(K, 64);
   p.kt = (int)ceil_div(K, 64 * kkb);
   p.tiles_p = (int)ceil_div(p.rows_p, kBM);
   p.tiles_q = 1;
@@ -1400,6 +1423,15 @@ nvfp4_status nvfp4_fused_proj(const uint8_t* a_codes, const uint8_t* a_scales, f
   if (!seg_offsets || !seg_global_scales || n_seg < 1 || n_seg > NVFP4_MAX_SEGMENTS) return NVFP4_ERR_INVALID_ARG;
   return run_gemm(a_codes, a_scales, a_global_scale, w_codes, w_scales, seg_offsets, seg_global_scales, n_seg, M,
                   seg_offsets[n_seg], K, out, out_dtype, (cudaStream_t)stream);
+}
+
+nvfp4_status nvfp4_mx_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* w_codes,
+                           const uint8_t* w_scales, int64_t M, int64_t N, int64_t K, void* out,
+                           nvfp4_out_dtype out_dtype, nvfp4_stream_t stream) {
+  const int64_t offs[2] = {0, N};
+  const float unit[1] = {1.0f};
+  return run_gemm(a_codes, a_scales, 1.0f, w_codes, w_scales, offs, unit, 1, M, N, K, out, out_dtype,
+                  (cudaStream_t)stream, /*mx=*/true);
 }
 
 nvfp4_status nvfp4_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_scales, float a_global_scale,

@@ -140,6 +140,22 @@ def test_harmonize_and_calibration_validation():
     assert L.nvfp4_amax_accumulate(A16, 0, 4, 64, P(0x10002), None) == nv.ERR_ALIGNMENT
 
 
+def test_mx_validation():
+    L = nv.lib()
+    assert L.nvfp4_mx_quantize(None, 0, 4, 64, A16, A16, 1, None) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_mx_quantize(A16, 0, 0, 64, A16, A16, 1, None) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_mx_quantize(A16, 0, 4, 48, A16, A16, 1, None) == nv.ERR_INVALID_ARG   # K % 32
+    assert L.nvfp4_mx_quantize(A16, 3, 4, 64, A16, A16, 1, None) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_mx_quantize(A16, 0, 4, 64, A16, A16, 2, None) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_mx_quantize(A1, 0, 4, 64, A16, A16, 1, None) == nv.ERR_ALIGNMENT
+    assert L.nvfp4_mx_quantize(A16, 0, 4, 64, A16, A1, 1, None) == nv.ERR_ALIGNMENT
+    assert L.nvfp4_mx_gemm(None, A16, A16, A16, 8, 16, 64, A16, 0, None) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_mx_gemm(A16, A16, A16, A16, 0, 16, 64, A16, 0, None) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_mx_gemm(A16, A16, A16, A16, 8, 16, 48, A16, 0, None) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_mx_gemm(A16, A16, A16, A16, 8, 16, 64, A16, 2, None) == nv.ERR_INVALID_ARG
+    assert L.nvfp4_mx_gemm(A16, A16, A1, A16, 8, 16, 64, A16, 0, None) == nv.ERR_ALIGNMENT
+
+
 def lin(x=A16, dt=0, M=8, K=64, ga=1.0, w=A16, sw=A16, gw=1.0, N=64, out=A16, od=0, ac=None, asc=None):
     return nv.lib().nvfp4_linear(x, dt, M, K, ctypes.c_float(ga), w, sw, ctypes.c_float(gw), N, out, od, ac, asc,
                                  None)
