@@ -14,7 +14,8 @@
 //
 // Work split: two threads per 32-element block, each owning 16 elements (the
 // NVFP4 quantizer's access pattern: two 16-byte loads of bf16 per thread, a
-// warp reads 1 KB); the pair combines its maxima with one shuffle.  HBM-bound:
+// warp reads 1 KB); the pair combines its maxima with one shuffle.  Each
+// thread keeps two such items in flight per iteration.  HBM-bound:
 // 2 + 0.5 + 1/32 bytes per bf16 element.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -42,39 +43,53 @@ __global__ void __launch_bounds__(256) mx_quantize_kernel(const void* __restrict
   const int lane = threadIdx.x & 31;
   const int64_t nblk = K / 32;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t wb = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); wb < total_items; wb += stride) {
-    const int64_t t = wb + lane;
-    const bool live = t < total_items;
-    const int64_t pb = t >> 1;
-    const int h = (int)(t & 1);
-    const int64_t r = pb / nblk_pad, j = pb - r * nblk_pad;
-    const bool real = live && r < M && j < nblk;
-    float f[16];
-    float amax = 0.0f;
-    if (real) {
-      Block16<kF32> B;
-      load_block<kF32>(x, (uint32_t)(r * (K / 16) + 2 * j + h), B);
-      amax = block_amax<kF32>(B);
-      block_floats<kF32>(B, f);
-    }
-    amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-    if (!live) continue;
-    const uint32_t ef = __float_as_uint(amax) >> 23;        // amax >= 0: the exponent field
-    const uint32_t sbyte = ef >= 2 ? ef - 2 : 0;             // E + 127
-    if (real) {
-      const float inv = __uint_as_float((254u - sbyte) << 23);  // 2^-E, normal for every byte produced
-      float lo[8], hi[8];
+  // two work items per thread per iteration, both loads issued first
+  for (int64_t wb = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); wb < total_items; wb += 2 * stride) {
+    Block16<kF32> B[2];
+    bool real[2], live[2];
+    int64_t r[2], j[2];
+    int h[2];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        lo[i] = f[i] * inv;
-        hi[i] = f[8 + i] * inv;
-      }
-      *reinterpret_cast<uint2*>(codes + r * (K / 2) + j * 16 + h * 8) = make_uint2(cvt_e2m1x8(lo), cvt_e2m1x8(hi));
+    for (int u = 0; u < 2; ++u) {
+      const int64_t t = wb + u * stride + lane;
+      live[u] = t < total_items;
+      const int64_t pb = t >> 1;
+      h[u] = (int)(t & 1);
+      r[u] = pb / nblk_pad;
+      j[u] = pb - r[u] * nblk_pad;
+      real[u] = live[u] && r[u] < M && j[u] < nblk;
+      if (real[u]) load_block<kF32>(x, (uint32_t)(r[u] * (K / 16) + 2 * j[u] + h[u]), B[u]);
     }
-    if (h == 0) {
-      const int64_t off = kTC ? ((r >> 7) * kc + (j >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (j & 3)
-                              : r * nblk + j;
-      scales[off] = real ? (uint8_t)sbyte : (uint8_t)0;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (wb + u * stride >= total_items) break;          // warp-uniform
+      float f[16];
+      float amax = 0.0f;
+      if (real[u]) {
+        amax = block_amax<kF32>(B[u]);
+        block_floats<kF32>(B[u], f);
+      }
+      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+      if (!live[u]) continue;
+      const uint32_t ef = __float_as_uint(amax) >> 23;        // amax >= 0: the exponent field
+      const uint32_t sbyte = ef >= 2 ? ef - 2 : 0;             // E + 127
+      if (real[u]) {
+        const float inv = __uint_as_float((254u - sbyte) << 23);  // 2^-E, normal for every byte produced
+        float lo[8], hi[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          lo[i] = f[i] * inv;
+          hi[i] = f[8 + i] * inv;
+        }
+        *reinterpret_cast<uint2*>(codes + r[u] * (K / 2) + j[u] * 16 + h[u] * 8) =
+            make_uint2(cvt_e2m1x8(lo), cvt_e2m1x8(hi));
+      }
+      if (h[u] == 0) {
+        const int64_t off = kTC ? ((r[u] >> 7) * kc + (j[u] >> 2)) * 512 + (r[u] & 31) * 16 + ((r[u] >> 5) & 3) * 4 +
+                                      (j[u] & 3)
+                                : r[u] * nblk + j[u];
+        scales[off] = real[u] ? (uint8_t)sbyte : (uint8_t)0;
+      }
     }
   }
 }
@@ -99,7 +114,7 @@ nvfp4_status nvfp4_mx_quantize(const void* x, nvfp4_in_dtype dtype, int64_t M, i
   const int64_t rows = tc ? ceil_div(M, 128) * 128 : M;
   const int64_t nblk_pad = tc ? 4 * kc : K / 32;
   const int64_t total = rows * nblk_pad * 2;
-  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(total, 256), (int64_t)d->sm_count * 4));
+  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(total, 512), (int64_t)d->sm_count * 4));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(blocks);
   cfg.blockDim = dim3(256);
