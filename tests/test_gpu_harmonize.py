@@ -113,3 +113,33 @@ def test_single_scale_gemm_on_harmonized_weights():
         assert e_h < 0.05, (i, e_h)          # half an E4M3 step per scale at most
         if i > 0:
             assert e_b > 1.0, (i, e_b)       # g_i / g_0 is 4 or more there
+
+
+def test_cases_where_the_fp32_order_decides():
+    """Ratios that put s * g / g_i next to an E4M3 rounding midpoint, where
+    rounding g / g_i to FP32 first and rounding once at the end disagree
+    (found on the CPU); the kernel must take the oracle's FP32 order."""
+    vals = torch.arange(1, 0x7F, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy()
+    rng = np.random.default_rng(61)
+    found = 0
+    for _ in range(20000):
+        v = float(vals[rng.integers(len(vals))])
+        k = int(rng.integers(0, len(vals) - 1))
+        if vals[k + 1] > v:
+            continue
+        mid = (float(vals[k]) + float(vals[k + 1])) / 2
+        g_i = np.float32(rng.uniform(1, 4000))
+        g = np.float32(np.float32(mid / v) * g_i)
+        byte = int(torch.tensor(np.float32(v)).to(torch.float8_e4m3fn).view(torch.uint8))
+        sc = np.full((1, 2), byte, np.uint8)                # N = 1, K = 32
+        want = oracle.harmonize_scales(sc, [0, 1], [g_i], g)
+        exact = np.float32(v * float(g) / float(g_i))       # double product, one rounding
+        if want[0, 0] == int(torch.tensor(exact).to(torch.float8_e4m3fn).view(torch.uint8)):
+            continue
+        for layout in (nv.SF_ROWMAJOR, nv.SF_TCGEN05):
+            got = _gpu_harmonize(sc, 32, [0, 1], [g_i], g, layout)
+            assert np.array_equal(got, _expect(sc, 32, [0, 1], [g_i], g, layout)), (v, g_i, g, layout)
+        found += 1
+        if found == 12:
+            break
+    assert found == 12

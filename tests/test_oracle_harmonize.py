@@ -130,3 +130,35 @@ def test_one_weight_scale_for_all_segments_scales_segment_i_by_g_i_over_g_0():
         # FP64 sums in another order: compare against the segment's scale
         np.testing.assert_allclose(broken[:, seg], want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
     assert float(gs[3]) / float(gs[0]) > 20  # the last segments come out far too large
+
+
+def test_the_fp32_order_decides_near_e4m3_midpoints():
+    """Cases where s * g / g_i lands next to an E4M3 rounding midpoint, so
+    that rounding g / g_i to FP32 first (the reading taken) and rounding the
+    exact product once give different bytes; the oracle must give the first,
+    as torch's cast of the FP32 product does."""
+    from fractions import Fraction
+
+    vals = torch.arange(1, 0x7F, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy()
+    cast = lambda y: int(torch.tensor(np.float32(y)).to(torch.float8_e4m3fn).view(torch.uint8))  # noqa: E731
+    rng = np.random.default_rng(60)
+    found = 0
+    for _ in range(20000):
+        v = float(vals[rng.integers(len(vals))])
+        k = int(rng.integers(0, len(vals) - 1))
+        if vals[k + 1] > v:
+            continue
+        mid = (float(vals[k]) + float(vals[k + 1])) / 2
+        g_i = np.float32(rng.uniform(1, 4000))
+        g = np.float32(np.float32(mid / v) * g_i)
+        fp32_order = cast(np.float32(np.float32(v) * np.float32(g / g_i)))
+        exact_order = cast(float(Fraction(v) * Fraction(float(g)) / Fraction(float(g_i))))
+        if fp32_order == exact_order:
+            continue
+        byte = np.uint8(cast(v))
+        out = oracle.harmonize_scales(np.full((1, 2), byte, np.uint8), [0, 1], [g_i], g)
+        assert out[0, 0] == fp32_order and out[0, 1] == fp32_order, (v, g_i, g)
+        found += 1
+        if found == 12:
+            break
+    assert found == 12
