@@ -137,8 +137,10 @@ class ClockSampler:
         if self.t is not None:
             self.t.join(timeout=2)
 
-    def summary(self, t0: float, t1: float):
-        rows = [l for (t, l) in self.lines if t0 - 0.25 <= t <= t1 + 0.25] or [l for (_, l) in self.lines]
+    def summary(self, t0: float, t1: float, strict: bool = False):
+        rows = [l for (t, l) in self.lines if t0 - 0.25 <= t <= t1 + 0.25]
+        if not rows and not strict:
+            rows = [l for (_, l) in self.lines]
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
@@ -364,6 +366,21 @@ def time_eager(torch, fn, steps, warmup):
     return start.elapsed_time(end) / steps
 
 
+def soak_clocks(torch, graph, ms_per_replay, stream, sampler, seconds=1.0):
+    """Replay a captured graph back to back for about `seconds` (untimed) and
+    return the clock samples of that window, or None without samples."""
+    if sampler is None or graph is None:
+        return None
+    n = max(1, int(seconds / max(ms_per_replay * 1e-3, 1e-6)))
+    torch.cuda.synchronize()
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        for _ in range(n):
+            graph.replay()
+    torch.cuda.synchronize()
+    return sampler.summary(t0, time.time(), strict=True)
+
+
 # ----------------------------------------------------------------- CPU oracle
 
 def oracle_decode_sample(budget_s=12.0, max_steps=40, warmup=0, exact=False):
@@ -507,7 +524,7 @@ def measure_decode(torch, nv, synth, dev, rank, world, l2, args, stream, barrier
     return line, t_soak, t_end
 
 
-def measure_prefill(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind):
+def measure_prefill(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind, sampler=None):
     w = synth.PREFILL
     if args.prefill_m:
         import dataclasses
@@ -517,6 +534,7 @@ def measure_prefill(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_k
     with torch.cuda.stream(stream):
         ms_p, g1 = time_graph(torch, p.step, k, 3, stream)
         ms_pg, g2 = time_graph(torch, p.gemm_only, k, 3, stream)
+    clk = soak_clocks(torch, g2, ms_pg * k, stream, sampler)
     del g1, g2
     fp4_peak = float(peaks["bf16_tflops"]) * FP4_OVER_BF16
     fp4_sust = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])) * FP4_OVER_BF16
@@ -530,7 +548,8 @@ def measure_prefill(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_k
                      "peak_kind": f"{peak_kind} bf16 cuBLAS x {FP4_OVER_BF16:g} (nominal fp4/bf16)",
                      "flops_per_launch": p.flops, "ms_per_launch": ms_pg,
                      "traffic": profiled_traffic("nvfp4_gemm_kernel", "prefill")},
-        "l2": "inputs 129 MB + 1.14 GB output per step exceed L2"}
+        "l2": "inputs 129 MB + 1.14 GB output per step exceed L2",
+        "clocks_gemm_back_to_back": clk}
     del p
     nv.nvfp4_forget_static()
     return res
@@ -669,7 +688,7 @@ def measure_harmonize(torch, nv, synth, dev, rank, l2, args, stream, peaks):
     return res
 
 
-def measure_mx(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind):
+def measure_mx(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind, sampler=None):
     """MXFP4, the contrast format: its quantizer (X[4096,5120] bf16), its
     kind::mxf4 GEMM on the prefill and decode shapes (weights rotated through
     copies larger than L2), and the GEMM error of NVFP4 and MXFP4 against the
@@ -709,12 +728,15 @@ def measure_mx(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind):
     def gp(i):
         nv.nvfp4_mx_gemm(ac, as_, wc, ws, pm, w.N, w.K, out)
 
+    kp = max(3, min(args.steps, 10))
     with torch.cuda.stream(stream):
-        ms_p, g2 = time_graph(torch, gp, max(3, min(args.steps, 10)), 3, stream)
+        ms_p, g2 = time_graph(torch, gp, kp, 3, stream)
+    clk = soak_clocks(torch, g2, ms_p * kp, stream, sampler)
     del g2
     fl = 2.0 * pm * w.N * w.K
     res["gemm_prefill"] = {"shape": [pm, w.N, w.K], "ms": ms_p, "TFLOP/s": fl / (ms_p * 1e-3) / 1e12,
-                           "frac_fp4_peak": fl / (ms_p * 1e-3) / 1e12 / tc_peak, "peak": peak_kind}
+                           "frac_fp4_peak": fl / (ms_p * 1e-3) / 1e12 / tc_peak, "peak": peak_kind,
+                           "clocks_gemm_back_to_back": clk}
     del ac, as_, wc, ws, out
     # decode-shape GEMM
     d = synth.DECODE
@@ -823,7 +845,7 @@ def main():
             res, _, _ = measure_decode(torch, nv, synth, dev, rank, world, l2, args, stream, barrier,
                                        max_over_ranks, peaks, peak_kind)
         elif args.only == "prefill":
-            res = measure_prefill(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind)
+            res = measure_prefill(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind, sampler)
         elif args.only == "fused":
             res = measure_fused(torch, nv, synth, dev, rank, l2, args, stream)
         elif args.only == "calib":
@@ -831,7 +853,7 @@ def main():
         elif args.only == "harmonize":
             res = measure_harmonize(torch, nv, synth, dev, rank, l2, args, stream, peaks)
         elif args.only == "mx":
-            res = measure_mx(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind)
+            res = measure_mx(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind, sampler)
         else:
             res = measure_quant_sweep(torch, nv, synth, dev, args, stream, peaks)
         sampler.stop()
@@ -843,12 +865,12 @@ def main():
     clk = sampler.summary(t_soak, t_end)
     if not args.no_extra and world == 1:
         line["extra"] = {
-            "prefill": measure_prefill(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind),
+            "prefill": measure_prefill(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind, sampler),
             "fused_gdn": measure_fused(torch, nv, synth, dev, rank, l2, args, stream),
             "quantize_sweep": measure_quant_sweep(torch, nv, synth, dev, args, stream, peaks),
             "static_calibration": measure_calibration(torch, nv, synth, dev, args, stream, peaks),
             "harmonize": measure_harmonize(torch, nv, synth, dev, rank, l2, args, stream, peaks),
-            "mxfp4": measure_mx(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind),
+            "mxfp4": measure_mx(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind, sampler),
         }
     sampler.stop()
     if clk is not None:
