@@ -207,6 +207,26 @@ NVFP4_API nvfp4_status nvfp4_linear(const void* x, nvfp4_in_dtype x_dtype, int64
                           float w_global_scale, int64_t N, void* out, nvfp4_out_dtype out_dtype,
                           uint8_t* a_codes, uint8_t* a_scales, nvfp4_stream_t stream);
 
+/* The layer with host-resident activation and output, as one call: enqueues
+ * on `stream` the host-to-device copy of X into x_dev, nvfp4_linear(x_dev,
+ * ..., out_dev, ..., a_codes, a_scales) and the device-to-host copy of the
+ * result into out_host; returns once they are enqueued (synchronize the
+ * stream before reading out_host).  No counterpart in the pages: the serving
+ * form of the layer whose input and output live on the host.
+ *   x_host    host [M, K] bf16/f32, M*K elements; page-locked memory lets the
+ *             copy run asynchronously (pageable memory works, synchronously)
+ *   out_host  host [M, N] bf16/f32 per out_dtype
+ *   x_dev, out_dev  device staging buffers of the same sizes, 16-byte
+ *             aligned, owned by the caller; a_codes/a_scales as in
+ *             nvfp4_linear (may be NULL for its one-kernel decode form)
+ *   other arguments as nvfp4_linear.
+ * Errors: as nvfp4_linear; arguments are checked before anything is enqueued. */
+NVFP4_API nvfp4_status nvfp4_linear_host(const void* x_host, nvfp4_in_dtype x_dtype, int64_t M, int64_t K,
+                               float a_global_scale, const uint8_t* w_codes, const uint8_t* w_scales,
+                               float w_global_scale, int64_t N, void* out_host, nvfp4_out_dtype out_dtype,
+                               void* x_dev, uint8_t* a_codes, uint8_t* a_scales, void* out_dev,
+                               nvfp4_stream_t stream);
+
 /* nvfp4_gemm for decode-sized M that allocates nothing.  The pages have no
  * counterpart: this is an interface variant, not part of the method.  It
  * computes exactly what nvfp4_gemm computes for the same arguments (same

@@ -47,6 +47,8 @@ _lib.nvfp4_harmonize_scales.argtypes = [_vp, _i64, _i64, ctypes.c_int, ctypes.PO
                                         ctypes.c_int, _f32, _vp, _vp]
 _lib.nvfp4_mx_quantize.argtypes = [_vp, ctypes.c_int, _i64, _i64, _vp, _vp, ctypes.c_int, _vp]
 _lib.nvfp4_mx_gemm.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, ctypes.c_int, _vp]
+_lib.nvfp4_linear_host.argtypes = [_vp, ctypes.c_int, _i64, _i64, _f32, _vp, _vp, _f32, _i64, _vp, ctypes.c_int, _vp,
+                                   _vp, _vp, _vp, _vp]
 _lib.nvfp4_quantize.argtypes = [_vp, ctypes.c_int, _i64, _i64, _f32, _vp, _vp, ctypes.c_int, _vp, _vp]
 _lib.nvfp4_swizzle_scales.argtypes = [_vp, _i64, _i64, _vp, _vp]
 _lib.nvfp4_gemm.argtypes = [_vp, _vp, _f32, _vp, _vp, _f32, _i64, _i64, _i64, _vp, ctypes.c_int, _vp]
@@ -108,6 +110,14 @@ def _ptr(t):
         return None
     if not t.is_cuda:
         raise ValueError("device tensor expected")
+    if not t.is_contiguous():
+        raise ValueError("contiguous tensor expected")
+    return _vp(t.data_ptr())
+
+
+def _hptr(t: torch.Tensor):
+    if t.is_cuda:
+        raise ValueError("host tensor expected")
     if not t.is_contiguous():
         raise ValueError("contiguous tensor expected")
     return _vp(t.data_ptr())
@@ -181,6 +191,20 @@ def nvfp4_linear(x: torch.Tensor, a_global_scale, w_codes, w_scales, w_global_sc
                              float(w_global_scale), N, _ptr(out), _out_dtype(out),
                              _ptr(a_codes) if a_codes is not None else None,
                              _ptr(a_scales) if a_scales is not None else None, _stream(out)))
+
+
+def nvfp4_linear_host(x_host: torch.Tensor, a_global_scale, w_codes, w_scales, w_global_scale, N,
+                      out_host: torch.Tensor, x_dev: torch.Tensor, out_dev: torch.Tensor, a_codes=None,
+                      a_scales=None) -> None:
+    """x_host / out_host: CPU tensors (page-locked for asynchronous copies);
+    x_dev / out_dev: device staging tensors of the same shapes and dtypes."""
+    M, K = x_host.shape
+    _check("nvfp4_linear_host",
+           _lib.nvfp4_linear_host(_hptr(x_host), _in_dtype(x_host), M, K, float(a_global_scale), _ptr(w_codes),
+                                  _ptr(w_scales), float(w_global_scale), N, _hptr(out_host), _out_dtype(out_host),
+                                  _ptr(x_dev), _ptr(a_codes) if a_codes is not None else None,
+                                  _ptr(a_scales) if a_scales is not None else None, _ptr(out_dev),
+                                  _stream(out_dev)))
 
 
 def nvfp4_gemm_noalloc(a_codes, a_scales, a_global_scale, w_codes, w_scales, w_global_scale, M, N, K,

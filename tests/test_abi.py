@@ -176,6 +176,25 @@ def test_linear_validation():
     assert lin(sw=A1) == nv.ERR_ALIGNMENT
 
 
+def test_linear_host_validation():
+    L = nv.lib()
+
+    def lh(xh=A16, dt=0, M=8, K=64, ga=1.0, w=A16, sw=A16, gw=1.0, N=64, oh=A16, od=0, xd=A16, od_=A16):
+        return L.nvfp4_linear_host(xh, dt, M, K, ctypes.c_float(ga), w, sw, ctypes.c_float(gw), N, oh, od, xd, None,
+                                   None, od_, None)
+    assert lh(xh=None) == nv.ERR_INVALID_ARG
+    assert lh(oh=None) == nv.ERR_INVALID_ARG
+    assert lh(xd=None) == nv.ERR_INVALID_ARG
+    assert lh(od_=None) == nv.ERR_INVALID_ARG
+    assert lh(M=0) == nv.ERR_INVALID_ARG
+    assert lh(K=48) == nv.ERR_INVALID_ARG
+    assert lh(dt=2) == nv.ERR_INVALID_ARG
+    assert lh(od=2) == nv.ERR_INVALID_ARG
+    assert lh(ga=0.0) == nv.ERR_INVALID_ARG
+    assert lh(xd=A1) == nv.ERR_ALIGNMENT
+    assert lh(od_=A1) == nv.ERR_ALIGNMENT
+
+
 def test_declare_static_validation():
     L = nv.lib()
     assert L.nvfp4_declare_static(None, 64) == nv.ERR_INVALID_ARG

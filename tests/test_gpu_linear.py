@@ -111,3 +111,24 @@ def test_linear_chain_reads_the_previous_layers_output():
         torch.cuda.synchronize()
         assert torch.equal(h, h_ref) and torch.equal(y, y_ref)
     check_device_error_word()
+
+
+@pytest.mark.parametrize("M,N,K,buffers,pinned", [(8, 12288, 5120, True, True), (8, 12288, 5120, False, True),
+                                                  (64, 1024, 2048, True, False), (5, 1000, 320, False, False)])
+def test_linear_host_equals_the_device_call(M, N, K, buffers, pinned):
+    x = synth.student_t_outliers(M, K, seed=M + N, dtype=torch.bfloat16)
+    wcd, wsd, gw, _ = _weights(N, K, seed=K + 1)
+    ga = float(oracle.global_scale(oracle.amax(x.float().numpy())))
+    x_host = x.pin_memory() if pinned else x.clone()
+    out_host = torch.full((M, N), float("nan"), dtype=torch.bfloat16)
+    if pinned:
+        out_host = out_host.pin_memory()
+    x_dev = torch.empty(M, K, dtype=torch.bfloat16, device=DEV)
+    out_dev = torch.empty(M, N, dtype=torch.bfloat16, device=DEV)
+    ac, asc = nv.alloc_quantized(M, K, DEV) if buffers else (None, None)
+    nv.nvfp4_linear_host(x_host, ga, wcd, wsd, gw, N, out_host, x_dev, out_dev, ac, asc)
+    torch.cuda.synchronize()
+    check_device_error_word()
+    want = _two_kernels(x.to(DEV), ga, wcd, wsd, gw, N, torch.bfloat16)
+    torch.cuda.synchronize()
+    assert torch.equal(out_host, want.cpu())
