@@ -18,11 +18,18 @@
  *      [anthology record LIT-800, "Standing in the anthology"; cctest.ai
  *      article, "Main findings"; podcast abstract].
  *
+ * Around them: the offline rewrite of a fused weight's scales to one common
+ * global scale (the "pre-harmonized" checkpoint), the running amax of a
+ * static calibration, and the MXFP4 format the pages contrast NVFP4 with
+ * (32-element blocks, power-of-two scales): its quantizer and GEMM.
+ *
  * Conventions shared by every entry point
  *   - Device pointers are raw CUDA device addresses owned by the caller; the
  *     library never allocates, frees or retains them.  Host pointers (named
- *     so below) are read during the call only.  The one buffer the library
- *     owns is the GEMM's K-split workspace (see nvfp4_gemm).
+ *     so below) are read during the call only, except the buffers of
+ *     nvfp4_linear_host, which its enqueued copies use until the stream
+ *     reaches them.  The one buffer the library owns is the GEMM's K-split
+ *     workspace (see nvfp4_gemm).
  *   - Consecutive kernels of this library on one stream overlap their
  *     prologue with the previous kernel's tail (programmatic dependent
  *     launch); each still reads its inputs only after the kernel before it
