@@ -9,6 +9,7 @@ codes E2M1(x / 2^E), nearest even, saturating.
 
 What fixes it, other than the oracle itself:
   * hand-derived blocks (scale byte and codes worked out by hand);
+  * torch's float8_e8m0fnu decoding of every finite scale byte;
   * Python's frexp for floor(log2 amax), and amax / 2^E in [4, 8);
   * brute force over the E2M1 values in exact rational arithmetic;
   * the exact rational GEMM sum on small operands, numpy's FP64 matmul on
@@ -132,3 +133,11 @@ def test_sixteen_element_blocks_keep_outliers_local():
         mc, ms = oracle.mx_quantize(x)
         e_mx = np.linalg.norm(oracle.mx_dequantize(mc, ms) - x) / np.linalg.norm(x)
         assert e_nv < 0.85 * e_mx, (e_nv, e_mx)
+
+
+def test_e8m0_decode_matches_torch():
+    """torch's float8_e8m0fnu (the OCP E8M0 scale type) decodes every finite
+    byte to the same power of two."""
+    t = torch.arange(0, 255, dtype=torch.uint8).view(torch.float8_e8m0fnu).float().double().numpy()
+    for b in range(255):
+        assert oracle.e8m0_decode(b) == t[b], b
