@@ -310,26 +310,41 @@ class FusedGDN:
 
 
 class QuantSweep:
-    def __init__(self, torch, nv, synth, dev, M, K):
+    """One point of the quantize sweep.  Where X is smaller than the L2, the
+    step rotates through copies of X (and of the outputs) totalling more
+    than 3x the L2 (at most 16 copies), so no step finds its input in L2;
+    the M <= 64 points are latency-bound and use at most 16 copies."""
+
+    MAX_COPIES = 16
+
+    def __init__(self, torch, nv, synth, dev, M, K, l2_bytes):
         self.nv = nv
-        self.x = synth.quant_sweep_activation(M, K, device=dev)
+        x = synth.quant_sweep_activation(M, K, device=dev)
         self.M, self.K = M, K
-        self.codes, self.sc = nv.alloc_quantized(M, K, dev)
-        self.am = torch.empty(1, dtype=torch.float32, device=dev)
-        nv.nvfp4_amax(self.x, self.am)
-        self.g = 2688.0 / self.am.item()
         self.bytes = M * K * 2 + M * K // 2 + M * K // 16
+        self.n_copies = max(1, min(self.MAX_COPIES, math.ceil(3 * l2_bytes / self.bytes)))
+        self.xs = [x] + [x.clone() for _ in range(self.n_copies - 1)]
+        self.outs = [nv.alloc_quantized(M, K, dev) for _ in range(self.n_copies)]
+        self.am = torch.empty(1, dtype=torch.float32, device=dev)
+        nv.nvfp4_amax(x, self.am)
+        self.g = 2688.0 / self.am.item()
 
     def step(self, i):
-        self.nv.nvfp4_quantize(self.x, self.g, self.codes, self.sc, self.nv.SF_TCGEN05, self.am)
+        j = i % self.n_copies
+        codes, sc = self.outs[j]
+        self.nv.nvfp4_quantize(self.xs[j], self.g, codes, sc, self.nv.SF_TCGEN05, self.am)
 
 
 # ----------------------------------------------------------------- timing
 
-def time_graph(torch, fn, steps, warmup, stream, flush=None):
-    """Warm up eagerly, capture `steps` calls of fn(i) in one CUDA graph,
-    replay once untimed, then time one replay with events on `stream`.
-    Returns (ms per step, graph)."""
+REPLAYS = 10     # timed replays of each captured graph; the median is reported
+
+
+def time_graph(torch, fn, steps, warmup, stream, replays=REPLAYS):
+    """Warm up eagerly, capture `steps` calls of fn(i) in one CUDA graph and
+    replay it once untimed; then replay it `replays` times back to back, each
+    replay bracketed by CUDA events on `stream`.  Returns (median over the
+    replays of ms per step, graph)."""
     for i in range(warmup):
         fn(i)
     torch.cuda.synchronize()
@@ -339,16 +354,14 @@ def time_graph(torch, fn, steps, warmup, stream, flush=None):
             fn(i)
     g.replay()
     torch.cuda.synchronize()
-    if flush is not None:
-        flush()
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    start.record(stream)
-    g.replay()
-    end.record(stream)
-    end.synchronize()
-    return start.elapsed_time(end) / steps, g
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(replays)]
+    for start, end in evs:
+        start.record(stream)
+        g.replay()
+        end.record(stream)
+    evs[-1][1].synchronize()
+    per_step = sorted(start.elapsed_time(end) / steps for start, end in evs)
+    return statistics.median(per_step), g
 
 
 def time_eager(torch, fn, steps, warmup):
@@ -512,7 +525,9 @@ def measure_decode(torch, nv, synth, dev, rank, world, l2, args, stream, barrier
         "e2e": {"value": world * d.step_bytes / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
                 "ms_per_step": ms_e2e, "h2d_bytes_per_step": d.x.numel() * d.x.element_size(),
                 "d2h_bytes_per_step": d.out.numel() * d.out.element_size()},
-        "gpu_launches": d.launches_per_step * args.steps,
+        "timing": f"median over {REPLAYS} back-to-back replays of a CUDA graph of K steps, CUDA events on the "
+                  f"launching stream; every replay is inside the timed region",
+        "gpu_launches": d.launches_per_step * args.steps * REPLAYS,
         "decode_one_kernel": {
             "step": "nvfp4_linear without activation buffers: one kernel quantizes X in shared memory",
             "ms_per_step": ms_one, "GB/s": world * d.layer_bytes / (ms_one * 1e-3) / 1e9,
@@ -521,6 +536,19 @@ def measure_decode(torch, nv, synth, dev, rank, world, l2, args, stream, barrier
     del d
     nv.nvfp4_forget_static()
     return line, t_soak, t_end
+
+
+def tensor_roofline(kernel, flops, ms, peaks, peak_kind, traffic):
+    """Roofline record of a tensor-bound launch against the dense FP4 peak
+    (measured BF16 burst x the nominal FP4 : BF16 ratio), with the
+    sustained-clock figure beside it."""
+    fp4_peak = float(peaks["bf16_tflops"]) * FP4_OVER_BF16
+    fp4_sust = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])) * FP4_OVER_BF16
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"bound": "tensor", "kernel": kernel, "flops_per_launch": flops, "ms_per_launch": ms,
+            "peak_kind": f"{peak_kind} bf16 cuBLAS x {FP4_OVER_BF16:g} (nominal fp4/bf16)",
+            "traffic": traffic, "frac_of_sustained": round(tf / fp4_sust, 4), "unit": "TFLOP/s",
+            "peak": fp4_peak, "achieved": round(tf, 1), "frac": round(tf / fp4_peak, 4)}
 
 
 def measure_prefill(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind, sampler=None):
@@ -535,52 +563,65 @@ def measure_prefill(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_k
         ms_pg, g2 = time_graph(torch, p.gemm_only, k, 3, stream)
     clk = soak_clocks(torch, g2, ms_pg * k, stream, sampler)
     del g1, g2
-    fp4_peak = float(peaks["bf16_tflops"]) * FP4_OVER_BF16
-    fp4_sust = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])) * FP4_OVER_BF16
-    tf = p.flops / (ms_pg * 1e-3) / 1e12
     res = {
-        "workload": f"prefill-shape linear X[{w.M},5120] bf16 x W[17408,5120] nvfp4 -> bf16",
-        "step_tflops": p.flops / (ms_p * 1e-3) / 1e12, "ms_per_step": ms_p,
-        "roofline": {"bound": "tensor", "kernel": "nvfp4_gemm_kernel<256>", "achieved": tf,
-                     "peak": fp4_peak, "unit": "TFLOP/s", "frac": tf / fp4_peak,
-                     "frac_of_sustained": tf / fp4_sust,
-                     "peak_kind": f"{peak_kind} bf16 cuBLAS x {FP4_OVER_BF16:g} (nominal fp4/bf16)",
-                     "flops_per_launch": p.flops, "ms_per_launch": ms_pg,
-                     "traffic": profiled_traffic("nvfp4_gemm_kernel", "prefill")},
-        "l2": "inputs 129 MB + 1.14 GB output per step exceed L2",
-        "clocks_gemm_back_to_back": clk}
+        "workload": f"prefill X[{w.M},5120] x W[17408,5120] nvfp4 -> bf16; inputs 129 MB + 1.14 GB output > L2",
+        "step": "quantize + GEMM", "ms_per_step": round(ms_p, 5),
+        "step_tflops": round(p.flops / (ms_p * 1e-3) / 1e12, 1),
+        "clocks_gemm_back_to_back": clk,
+        "roofline": tensor_roofline("nvfp4_gemm_kernel<256>", p.flops, ms_pg, peaks, peak_kind,
+                                    profiled_traffic("nvfp4_gemm_kernel", "prefill"))}
     del p
     nv.nvfp4_forget_static()
     return res
 
 
-def measure_fused(torch, nv, synth, dev, rank, l2, args, stream):
+def measure_fused(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind):
     f = FusedGDN(torch, nv, synth, dev, rank, l2)
     k = max(3, min(args.steps, 20))
+    w = f.w
+
+    def gemm_only(i):
+        f.nv.nvfp4_fused_proj(f.a_codes, f.a_sc, f.ga, f.wc, f.ws, f.offs, f.gs, w.M, w.K, f.out)
+
     with torch.cuda.stream(stream):
         ms_f, g3 = time_graph(torch, f.step, k, 3, stream)
-    del g3
-    res = {"workload": "fused GDN projection X[4096,5120] x W[8192|4096|48|48, 5120]",
-           "step_tflops": f.flops / (ms_f * 1e-3) / 1e12, "ms_per_step": ms_f}
+        ms_g, g4 = time_graph(torch, gemm_only, k, 3, stream)
+    del g3, g4
+    res = {"workload": "fused GDN projection X[4096,5120] x W[8192|4096|48|48, 5120], per-segment scales",
+           "step": "quantize + fused GEMM", "ms_per_step": round(ms_f, 5),
+           "step_tflops": round(f.flops / (ms_f * 1e-3) / 1e12, 1),
+           "roofline": tensor_roofline("nvfp4_gemm_kernel<256> (segment table)", f.flops, ms_g, peaks, peak_kind,
+                                       None)}
     del f
     nv.nvfp4_forget_static()
     return res
 
 
-def measure_quant_sweep(torch, nv, synth, dev, args, stream, peaks):
+def measure_mma_peak(nv, dev):
+    """The device's dense FP4 MMA throughput (context for the tensor
+    rooflines; the rooflines keep the measured BF16 x 4 denominator)."""
+    tf, per_clk = nv.nvfp4_measure_mma_peak(5000, dev)
+    return {"kernel": "mma_peak_kernel: 148 CTAs x 20,000 back-to-back tcgen05.mma kind::mxf4nvf4 "
+                      "128x256x64 from shared memory",
+            "TFLOP/s": round(tf, 1), "flop_per_clk_per_sm": round(per_clk, 1),
+            "at_1965_MHz_TFLOP/s": round(per_clk * 148 * 1.965e9 / 1e12, 1)}
+
+
+def measure_quant_sweep(torch, nv, synth, dev, args, stream, peaks, l2):
     hbm_peak = float(peaks["hbm_gbs"])
     sweep = {}
     for M in synth.QUANT_SWEEP_M:
         for K in synth.QUANT_SWEEP_K:
             if args.quant_point and args.quant_point != f"{M}x{K}":
                 continue
-            q = QuantSweep(torch, nv, synth, dev, M, K)
+            q = QuantSweep(torch, nv, synth, dev, M, K, l2)
             kk = max(3, min(args.steps, 50))
             with torch.cuda.stream(stream):
                 ms_q, g4 = time_graph(torch, q.step, kk, 3, stream)
             del g4
             gbs = q.bytes / (ms_q * 1e-3) / 1e9
-            sweep[f"{M}x{K}"] = {"us": ms_q * 1e3, "GB/s": gbs, "frac_hbm": gbs / hbm_peak}
+            sweep[f"{M}x{K}"] = {"us": round(ms_q * 1e3, 3), "GB/s": round(gbs, 1),
+                                 "frac_hbm": round(gbs / hbm_peak, 4), "x_copies": q.n_copies}
             del q
     return sweep
 
@@ -797,7 +838,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--only", default="all", choices=["all", "decode", "prefill", "fused", "quant", "calib", "harmonize", "mx"])
+    ap.add_argument("--only", default="all", choices=["all", "decode", "prefill", "fused", "quant", "calib", "harmonize", "mx",
+                                                      "peak"])
     ap.add_argument("--prefill-m", type=int, default=0, help="override M of the prefill workload")
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed decode steps first")
     ap.add_argument("--no-extra", action="store_true")
@@ -846,15 +888,17 @@ def main():
         elif args.only == "prefill":
             res = measure_prefill(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind, sampler)
         elif args.only == "fused":
-            res = measure_fused(torch, nv, synth, dev, rank, l2, args, stream)
+            res = measure_fused(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind)
         elif args.only == "calib":
             res = measure_calibration(torch, nv, synth, dev, args, stream, peaks)
         elif args.only == "harmonize":
             res = measure_harmonize(torch, nv, synth, dev, rank, l2, args, stream, peaks)
         elif args.only == "mx":
             res = measure_mx(torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind, sampler)
+        elif args.only == "peak":
+            res = measure_mma_peak(nv, dev)
         else:
-            res = measure_quant_sweep(torch, nv, synth, dev, args, stream, peaks)
+            res = measure_quant_sweep(torch, nv, synth, dev, args, stream, peaks, l2)
         sampler.stop()
         print(json.dumps({"only": args.only, "result": res}))
         return 0
@@ -862,6 +906,11 @@ def main():
     line, t_soak, t_end = measure_decode(torch, nv, synth, dev, rank, world, l2, args, stream, barrier,
                                          max_over_ranks, peaks, peak_kind)
     clk = sampler.summary(t_soak, t_end)
+    if clk is not None:
+        line["clocks"] = clk
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu, _, _ = oracle_decode_sample()
+        line["cpu_baseline"] = cpu
     if not args.no_extra and world == 1:
         def leg(fn, *a):
             # an extra workload that raises is reported as such; the headline
@@ -872,20 +921,19 @@ def main():
                 nv.nvfp4_forget_static()
                 return {"error": f"{type(e).__name__}: {e}"[:400]}
 
-        line["extra"] = {
-            "prefill": leg(measure_prefill, torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind, sampler),
-            "fused_gdn": leg(measure_fused, torch, nv, synth, dev, rank, l2, args, stream),
-            "quantize_sweep": leg(measure_quant_sweep, torch, nv, synth, dev, args, stream, peaks),
-            "static_calibration": leg(measure_calibration, torch, nv, synth, dev, args, stream, peaks),
-            "harmonize": leg(measure_harmonize, torch, nv, synth, dev, rank, l2, args, stream, peaks),
-            "mxfp4": leg(measure_mx, torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind, sampler),
-        }
+        # the tensor-bound rows come last, so that the end of the printed
+        # line (what a log tail keeps) carries them
+        extra = {}
+        extra["fp4_mma_peak"] = leg(measure_mma_peak, nv, dev)
+        extra["mxfp4"] = leg(measure_mx, torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind, sampler)
+        extra["harmonize"] = leg(measure_harmonize, torch, nv, synth, dev, rank, l2, args, stream, peaks)
+        extra["static_calibration"] = leg(measure_calibration, torch, nv, synth, dev, args, stream, peaks)
+        extra["quantize_sweep"] = leg(measure_quant_sweep, torch, nv, synth, dev, args, stream, peaks, l2)
+        extra["fused_gdn"] = leg(measure_fused, torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind)
+        extra["prefill"] = leg(measure_prefill, torch, nv, synth, dev, rank, l2, args, stream, peaks, peak_kind,
+                               sampler)
+        line["extra"] = extra
     sampler.stop()
-    if clk is not None:
-        line["clocks"] = clk
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu, _, _ = oracle_decode_sample()
-        line["cpu_baseline"] = cpu
     if rank == 0:
         print(json.dumps(line))
     if pg is not None:

@@ -28,8 +28,10 @@
  *     library never allocates, frees or retains them.  Host pointers (named
  *     so below) are read during the call only, except the buffers of
  *     nvfp4_linear_host, which its enqueued copies use until the stream
- *     reaches them.  The one buffer the library owns is the GEMM's K-split
- *     workspace (see nvfp4_gemm).
+ *     reaches them.  The one buffer the library may own is the GEMM's K-split
+ *     workspace of a stream, and only when the caller registered none for
+ *     that stream (see nvfp4_set_workspace); nvfp4_release_workspaces()
+ *     frees what it allocated.
  *   - Consecutive kernels of this library on one stream overlap their
  *     prologue with the previous kernel's tail (programmatic dependent
  *     launch); each still reads its inputs only after the kernel before it
@@ -163,19 +165,56 @@ NVFP4_API nvfp4_status nvfp4_swizzle_scales(const uint8_t* rowmajor, int64_t row
  * For M <= 128 (decode) the K loop of each weight tile is split across CTAs
  * so that every SM streams weight; the partial FP32 tiles are summed in a
  * fixed order (the result does not depend on timing and equals the unsplit
- * sum up to FP32 rounding order).  The partials go to a workspace the
- * library allocates on first use for each (device, stream) pair
- * (2 * SMs * 128 KB) and keeps until the process exits.  That first call on a
- * stream must not be made while the stream is being captured into a CUDA
- * graph: it returns UNSUPPORTED then.  Calls on one stream share its
- * workspace safely (stream order); calls on different streams use different
- * workspaces.
- * Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (device is not sm_100, or a
- * first decode-shaped call during capture), CUDA. */
+ * sum up to FP32 rounding order).  The partials go to the K-split workspace
+ * of (device, stream): the one the caller registered with
+ * nvfp4_set_workspace, else one the library allocates on the first such call
+ * on that stream (2 * SMs * 128 KB, zero-filled) and keeps until
+ * nvfp4_release_workspaces().  A library allocation cannot happen during
+ * CUDA graph capture: a first decode-shaped call on a capturing stream with
+ * no workspace returns UNSUPPORTED (register one, or make one call before
+ * capture).  Calls on one stream share its workspace safely (stream order);
+ * calls on different streams use different workspaces.  Each launch leaves
+ * the words it used empty (zero), so a workspace stays ready for the next.
+ * M > 128 uses no workspace.
+ * Errors: INVALID_ARG (also: a registered workspace smaller than
+ * nvfp4_workspace_bytes for this shape), ALIGNMENT, UNSUPPORTED (device is
+ * not sm_100, or a first decode-shaped call during capture with no
+ * workspace), CUDA. */
 NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float a_global_scale,
                         const uint8_t* w_codes, const uint8_t* w_scales, float w_global_scale,
                         int64_t M, int64_t N, int64_t K, void* out, nvfp4_out_dtype out_dtype,
                         nvfp4_stream_t stream);
+
+/* Bytes of K-split workspace nvfp4_gemm / nvfp4_linear need on the current
+ * device for an M x N x K problem: 2 * SMs * BN * 128 * 8, BN being the
+ * activation tile width the call picks (16, 32, 64 or 128 for M <= 16, 32,
+ * 64, 128); 0 for M > 128 (no split) or invalid sizes.  No counterpart in
+ * the pages: the sizing rule of this library's split-K exchange.
+ * nvfp4_workspace_bytes(128, N, K) (2 * SMs * 128 KB) covers every shape. */
+NVFP4_API size_t nvfp4_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* Register a caller-owned K-split workspace for `stream` on the current
+ * device; every later decode-shaped nvfp4_gemm / nvfp4_linear on that stream
+ * uses it instead of allocating.  No counterpart in the pages.
+ *   workspace  device memory, 16-byte aligned, at least
+ *              nvfp4_workspace_bytes(16, 1, 32) bytes, ZERO-FILLED when
+ *              registered (each launch leaves it zero again); owned by the
+ *              caller, who keeps it alive while calls that use it may run and
+ *              uses it for nothing else.  Calls whose shape needs more than
+ *              `bytes` return INVALID_ARG.
+ *   workspace NULL with bytes 0: unregister (the library allocates again on
+ *              the next decode-shaped call).
+ * A workspace the library had allocated for this stream is freed (after a
+ * device synchronize).  Registration is not stream-ordered: make it while no
+ * call on `stream` is in flight.
+ * Errors: INVALID_ARG (too small, or NULL with bytes != 0), ALIGNMENT, CUDA. */
+NVFP4_API nvfp4_status nvfp4_set_workspace(nvfp4_stream_t stream, void* workspace, size_t bytes);
+
+/* Free every K-split workspace the library allocated on the current device
+ * (after a device synchronize); registered ones are forgotten only by
+ * nvfp4_set_workspace(stream, NULL, 0).  Later calls allocate again.
+ * Errors: CUDA. */
+NVFP4_API nvfp4_status nvfp4_release_workspaces(void);
 
 /* Declare [base, base + bytes) read-only while library calls run (typically
  * the quantized weights of a model in serving).  No counterpart in the
@@ -237,9 +276,10 @@ NVFP4_API nvfp4_status nvfp4_linear_host(const void* x_host, nvfp4_in_dtype x_dt
 /* nvfp4_gemm for decode-sized M that allocates nothing.  The pages have no
  * counterpart: this is an interface variant, not part of the method.  It
  * computes exactly what nvfp4_gemm computes for the same arguments (same
- * kernel, same K split, same summation order), but the K-split partial tiles
- * and arrival counters live in a fixed scratch array in the library's static
- * device memory instead of a workspace allocated on first use.  For callers
+ * kernel, same K split, same summation order), but the K-split partial tiles,
+ * as tagged 64-bit words (an FP32 value and a "full" tag), live in a fixed
+ * scratch array in the library's static device memory instead of a workspace
+ * allocated on first use.  For callers
  * that must not allocate device memory once running (a serving engine that
  * plans its memory at start-up and gives the rest to its KV cache; code that
  * cannot take the implicit synchronisation of an allocation).
@@ -350,7 +390,10 @@ NVFP4_API nvfp4_status nvfp4_convert_e2m1(const float* in, uint8_t* out, int64_t
  * word: NVFP4_OK, NVFP4_ERR_TIMEOUT or NVFP4_ERR_DEVICE.  When the word was
  * set it also empties the GEMM's K-split scratch on this device (a launch that
  * gave up may leave partial tiles behind); GEMM results after a reported
- * error are reliable only once this call has returned. */
+ * error are reliable only once this call has returned.  The emptying runs
+ * after the synchronization: no GEMM may be enqueued on this device from
+ * another host thread while this call runs (its scratch words could be
+ * wiped mid-launch). */
 NVFP4_API nvfp4_status nvfp4_last_device_error(void);
 
 /* Bound (nanoseconds) on every wait inside this library's kernels on all
@@ -362,6 +405,35 @@ NVFP4_API void nvfp4_set_wait_timeout_ns(uint64_t ns);
  * records NVFP4_ERR_TIMEOUT in the device error word and exits; the context
  * stays usable.  Errors: INVALID_ARG (timeout_ns 0 or above 10 s), CUDA. */
 NVFP4_API nvfp4_status nvfp4_test_wait_timeout(uint64_t timeout_ns, nvfp4_stream_t stream);
+
+/* Test entry for the failure path of the decode GEMM's K split: runs
+ * nvfp4_gemm (noalloc = 0) or nvfp4_gemm_noalloc (noalloc != 0) on the same
+ * arguments, except that the CTA that sums each split weight tile never sees
+ * its helpers' partial tiles arrive.  Its bounded wait runs out (set the bound
+ * with nvfp4_set_wait_timeout_ns), it records NVFP4_ERR_TIMEOUT and skips that
+ * tile's output, and the helpers' partial words stay full in the scratch, as
+ * after a real timeout.  Output columns of split tiles are left unwritten.
+ * Errors: as the GEMM it runs; UNSUPPORTED for M > 128. */
+NVFP4_API nvfp4_status nvfp4_test_gemm_stalled_reduction(const uint8_t* a_codes, const uint8_t* a_scales,
+                                               float a_global_scale, const uint8_t* w_codes,
+                                               const uint8_t* w_scales, float w_global_scale, int64_t M,
+                                               int64_t N, int64_t K, void* out, nvfp4_out_dtype out_dtype,
+                                               int noalloc, nvfp4_stream_t stream);
+
+/* Measurement utility (no counterpart in the pages): the dense FP4
+ * tensor-core throughput of the current device.  One CTA per SM issues
+ * `iters` x 4 back-to-back tcgen05.mma kind::mxf4nvf4 block_scale
+ * (M = 128, N = 256, K = 64, E4M3 scales of 16-element blocks: the MMA the
+ * prefill GEMM issues) on operands resident in shared memory; a warm-up
+ * launch, then one launch timed with CUDA events on `stream`.  Synchronous.
+ *   tflops               host, written: 2*128*256*64 * 4*iters * SMs / time
+ *   flop_per_clk_per_sm  host, written: the same work per SM over the median
+ *                        SM's clock64 cycles (independent of the clock rate)
+ * 1 <= iters <= 2^20 (iters = 5000 runs for about 1.5 ms).
+ * Errors: INVALID_ARG, UNSUPPORTED (not sm_100, more than 1024 SMs), CUDA,
+ * TIMEOUT (a wait of the timed launch ran out). */
+NVFP4_API nvfp4_status nvfp4_measure_mma_peak(int iters, double* tflops, double* flop_per_clk_per_sm,
+                                              nvfp4_stream_t stream);
 
 /* Static description of a status code. */
 NVFP4_API const char* nvfp4_status_string(nvfp4_status status);

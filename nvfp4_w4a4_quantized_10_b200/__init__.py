@@ -53,6 +53,10 @@ _lib.nvfp4_quantize.argtypes = [_vp, ctypes.c_int, _i64, _i64, _f32, _vp, _vp, c
 _lib.nvfp4_swizzle_scales.argtypes = [_vp, _i64, _i64, _vp, _vp]
 _lib.nvfp4_gemm.argtypes = [_vp, _vp, _f32, _vp, _vp, _f32, _i64, _i64, _i64, _vp, ctypes.c_int, _vp]
 _lib.nvfp4_declare_static.argtypes = [_vp, ctypes.c_size_t]
+_lib.nvfp4_workspace_bytes.restype = ctypes.c_size_t
+_lib.nvfp4_workspace_bytes.argtypes = [_i64, _i64, _i64]
+_lib.nvfp4_set_workspace.argtypes = [_vp, _vp, ctypes.c_size_t]
+_lib.nvfp4_release_workspaces.argtypes = []
 _lib.nvfp4_forget_static.argtypes = []
 _lib.nvfp4_forget_static.restype = None
 _lib.nvfp4_linear.argtypes = [_vp, ctypes.c_int, _i64, _i64, _f32, _vp, _vp, _f32, _i64, _vp, ctypes.c_int, _vp, _vp,
@@ -66,6 +70,10 @@ _lib.nvfp4_last_device_error.argtypes = []
 _lib.nvfp4_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
 _lib.nvfp4_set_wait_timeout_ns.restype = None
 _lib.nvfp4_test_wait_timeout.argtypes = [ctypes.c_uint64, _vp]
+_lib.nvfp4_test_gemm_stalled_reduction.argtypes = [_vp, _vp, _f32, _vp, _vp, _f32, _i64, _i64, _i64, _vp,
+                                                   ctypes.c_int, ctypes.c_int, _vp]
+_lib.nvfp4_measure_mma_peak.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_double),
+                                        ctypes.POINTER(ctypes.c_double), _vp]
 _lib.nvfp4_status_string.restype = ctypes.c_char_p
 _lib.nvfp4_status_string.argtypes = [ctypes.c_int]
 _lib.nvfp4_version.restype = ctypes.c_int
@@ -179,6 +187,26 @@ def nvfp4_declare_static(t: torch.Tensor) -> None:
     _check("nvfp4_declare_static", _lib.nvfp4_declare_static(_ptr(t), t.numel() * t.element_size()))
 
 
+def nvfp4_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(_lib.nvfp4_workspace_bytes(M, N, K))
+
+
+def nvfp4_set_workspace(workspace, stream=None) -> None:
+    """Register a zero-filled uint8 device tensor as the K-split workspace of
+    `stream` (default: the tensor's current stream); None unregisters."""
+    if workspace is None:
+        st = torch.cuda.current_stream() if stream is None else stream
+        _check("nvfp4_set_workspace", _lib.nvfp4_set_workspace(_vp(st.cuda_stream), None, 0))
+        return
+    st = torch.cuda.current_stream(workspace.device) if stream is None else stream
+    _check("nvfp4_set_workspace",
+           _lib.nvfp4_set_workspace(_vp(st.cuda_stream), _ptr(workspace), workspace.numel() * workspace.element_size()))
+
+
+def nvfp4_release_workspaces() -> None:
+    _check("nvfp4_release_workspaces", _lib.nvfp4_release_workspaces())
+
+
 def nvfp4_forget_static() -> None:
     _lib.nvfp4_forget_static()
 
@@ -273,6 +301,24 @@ def nvfp4_test_wait_timeout(timeout_ns: int, device=None) -> None:
     dev = torch.device("cuda") if device is None else torch.device(device)
     _check("nvfp4_test_wait_timeout",
            _lib.nvfp4_test_wait_timeout(int(timeout_ns), _vp(torch.cuda.current_stream(dev).cuda_stream)))
+
+
+def nvfp4_test_gemm_stalled_reduction(a_codes, a_scales, a_global_scale, w_codes, w_scales, w_global_scale, M, N,
+                                      K, out: torch.Tensor, noalloc: bool = False) -> None:
+    _check("nvfp4_test_gemm_stalled_reduction",
+           _lib.nvfp4_test_gemm_stalled_reduction(_ptr(a_codes), _ptr(a_scales), float(a_global_scale),
+                                                  _ptr(w_codes), _ptr(w_scales), float(w_global_scale), M, N, K,
+                                                  _ptr(out), _out_dtype(out), int(bool(noalloc)), _stream(out)))
+
+
+def nvfp4_measure_mma_peak(iters: int = 5000, device=None):
+    """(TFLOP/s, FLOP per clock per SM) of back-to-back dense FP4 MMAs."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    tf, fc = ctypes.c_double(0.0), ctypes.c_double(0.0)
+    _check("nvfp4_measure_mma_peak",
+           _lib.nvfp4_measure_mma_peak(int(iters), ctypes.byref(tf), ctypes.byref(fc),
+                                       _vp(torch.cuda.current_stream(dev).cuda_stream)))
+    return tf.value, fc.value
 
 
 # ---------------------------------------------------------------- buffers

@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 SRC_DIR = os.path.join(HERE, "csrc")
 BUILD_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libnvfp4.so")
-SOURCES = ["runtime.cu", "quantize.cu", "gemm.cu", "harmonize.cu", "mxfp4.cu", "host_io.cu"]
+SOURCES = ["runtime.cu", "quantize.cu", "gemm.cu", "harmonize.cu", "mxfp4.cu", "host_io.cu", "mma_peak.cu"]
 HEADERS = ["ptx.cuh", "common.h", "block_quant.cuh", os.path.join("..", "..", "include", "nvfp4.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

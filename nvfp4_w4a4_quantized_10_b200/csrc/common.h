@@ -26,6 +26,12 @@ const DeviceInfo* device_info();
 // Wait bound for every kernel of the library (ns).
 uint64_t wait_timeout_ns();
 
+// Bound on a CTA's waits for its own in-flight copies and tensor-core work
+// before it frees shared memory and TMEM and exits: at least 1 s whatever the
+// wait bound above, so that a short wait bound (a test, or a caller that
+// wants quick failure reports) never lets a CTA exit under live copies.
+uint64_t drain_timeout_ns();
+
 // Empties every K-split scratch buffer of the GEMM on `device` (after a
 // device-side error left partial words behind).  Synchronous.
 cudaError_t clear_gemm_scratch(int device);

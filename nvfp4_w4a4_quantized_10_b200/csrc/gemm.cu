@@ -39,6 +39,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdio>
 #include <map>
 #include <mutex>
@@ -67,7 +68,8 @@ struct alignas(64) GemmParams {
   void* out;
   uint64_t* ws;          // swapped tiles: tagged FP32 partial tiles, 2 slots per CTA (all words empty between launches)
   unsigned* err;
-  uint64_t timeout_ns;
+  uint64_t timeout_ns;   // bound of every wait for work to arrive
+  uint64_t drain_ns;     // bound of the waits for a CTA's own copies and MMAs before it exits (>= 1 s)
   int64_t M, N;          // output [M, N]
   int rows_p, rows_q;    // rows of the P and Q operands
   int rb_q;              // 128-row scale blocks allocated for Q
@@ -78,6 +80,10 @@ struct alignas(64) GemmParams {
   int tma_store;         // 1: output through shared memory and TMA stores
   int w_static;          // 1: the weight lies in memory declared read-only (nvfp4_declare_static)
   int n_seg;
+  int test_stall;        // failure-path test only: the split-tile adder never sees its helpers' partials
+  int group_p;           // tile raster: P tiles per Q-tile sweep
+  CUtensorMap tmap_sfa;  // CTA pairs: scale chunks of P and Q as [chunks, 128] 32-bit words
+  CUtensorMap tmap_sfb;
   int seg_end[NVFP4_MAX_SEGMENTS];
   float seg_alpha[NVFP4_MAX_SEGMENTS];
   // activation quantized in the kernel (swapped tiles only): X [M, K]
@@ -93,7 +99,12 @@ struct alignas(64) GemmParams {
 // once, before the first MMA.
 // MX: MXFP4 operands (32-element blocks, E8M0 scales, kind::mxf4 with two
 // scales per MMA) instead of NVFP4 (16-element blocks, E4M3 scales).
-template <int BN, bool SWAP, int QX = 0, bool MX = false>
+// PAIR: prefill tiles of 256 x 256 computed by a pair of CTAs (a cluster of
+// two): each CTA loads its 128 activation rows and half of the 256 weight
+// rows (plus all 256 rows' scales); the even CTA issues the M = 256 MMAs and
+// scale copies for both (tcgen05 cta_group::2); each CTA drains its own 128
+// accumulator rows.
+template <int BN, bool SWAP, int QX = 0, bool MX = false, bool PAIR = false>
 struct Cfg {
   static constexpr bool kQx = QX != 0;
   // K per pipeline step: kKB blocks of 64 (one MMA each), 256 deep, as
@@ -107,7 +118,7 @@ struct Cfg {
   static constexpr uint32_t kSbo = 8 * kRowBytes;                    // bytes between 8-row groups
   static constexpr int kSfbBlocks = (BN + 127) / 128;                // 128-row scale blocks of Q
   static constexpr int kABytes = kBM * kRowBytes;
-  static constexpr int kBBytes = kQx ? 0 : BN * kRowBytes;           // Q codes per stage
+  static constexpr int kBBytes = kQx ? 0 : (PAIR ? BN / 2 : BN) * kRowBytes;   // Q codes per stage (per CTA)
   // scale chunks (128 rows x 4 scales, 512 bytes) per step: a chunk covers 64
   // K-elements of 16-element blocks (one MMA), or 128 of 32-element blocks
   static constexpr int kChunks = MX ? kKB / 2 : kKB;
@@ -122,7 +133,15 @@ struct Cfg {
   static constexpr int kActSfBytes = kKB * kSfChunk;
   static constexpr int kActBytes = kActSteps * (kActCodeBytes + kActSfBytes);
   static constexpr int kMaxStages = 8;
-  static constexpr int kFit = (222 * 1024 - kOutBytes - kActBytes) / kStageBytes;
+  // Decode tiles with a small activation side run two CTAs per SM: the next
+  // GEMM on the stream (programmatic dependent launch) then starts at once
+  // beside this one and streams its weight while this one finishes, instead
+  // of waiting for this grid's CTAs to leave.  Each CTA keeps to half of the
+  // SM's shared memory (and TMEM and registers).
+  static constexpr bool kCoRes = SWAP && !kQx && BN <= 32;
+  static constexpr int kMinBlocks = kCoRes ? 2 : 1;
+  static constexpr int kSmemBudget = kCoRes ? 112 * 1024 : 222 * 1024;
+  static constexpr int kFit = (kSmemBudget - kOutBytes - kActBytes) / kStageBytes;
   static constexpr int kStages = kFit < kMaxStages ? kFit : kMaxStages;
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + kStages * kABytes;
@@ -165,13 +184,18 @@ struct Cfg {
   static constexpr int kSfBase = kOverlapAcc ? kTmemCols - kSfRegions * kSfStageCols : kAccCols;
   static constexpr int kAcc1Col = kOverlapAcc ? kSfBase - 256 : 0;
   static constexpr int kSharedSlots = kOverlapAcc ? (256 - kAcc1Col + 63) / 64 : 0;   // drained before release
+  static constexpr int kTmemAlloc = kCoRes ? 256 : kTmemCols;         // columns this CTA allocates
   static_assert(kAcc1Col % 32 == 0, "accumulator column alignment");
   static_assert(kStages >= 2, "pipeline depth");
-  static_assert(kSfBase + kSfRegions * kSfStageCols <= kTmemCols, "TMEM budget");
+  static_assert(kSfBase + kSfRegions * kSfStageCols <= kTmemAlloc, "TMEM budget");
+  static_assert(!kCoRes || kSmemBytes <= 113 * 1024, "two CTAs per SM");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(BN % 16 == 0 && BN <= 256, "MMA N");
   static_assert(!kQx || (SWAP && BN <= 32), "in-kernel activation: swapped tiles, M <= 32");
   static_assert(!(kQx && MX), "in-kernel activation: NVFP4 only");
+  static_assert(!PAIR || (!SWAP && BN == 256 && !kQx), "CTA pairs: normal 256 x 256 tiles");
+  static constexpr int kMmaM = PAIR ? 2 * kBM : kBM;                 // MMA M (over the pair)
+  static constexpr int kGroupTiles = PAIR ? kGroupP / 2 : kGroupP;   // raster group, in tiles of P
   static_assert(kOffAct % 1024 == 0 && kActCodeBytes % 1024 == 0, "activation tiles on swizzle atoms");
 };
 
@@ -181,10 +205,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 __device__ __forceinline__ void tile_coords(const GemmParams& p, int tile, int& tp, int& tq) {
-  const int per_group = kGroupP * p.tiles_q;
+  const int per_group = p.group_p * p.tiles_q;
   const int group = tile / per_group;
-  const int first = group * kGroupP;
-  const int gsize = min(p.tiles_p - first, kGroupP);
+  const int first = group * p.group_p;
+  const int gsize = min(p.tiles_p - first, p.group_p);
   const int local = tile - group * per_group;
   tp = first + local % gsize;
   tq = local / gsize;
@@ -196,10 +220,12 @@ __device__ __forceinline__ void tile_coords(const GemmParams& p, int tile, int& 
 //   into gridDim.x contiguous, balanced ranges; CTA c owns units
 //   [floor(c U / G), floor((c+1) U / G)).  An item is the part of that range
 //   inside one tile.
+//   CTA pairs: whole 256 x 256 tiles t = pair, pair + pairs, ... for the
+//   pair index blockIdx.x / 2.
 struct WorkIter {
   int64_t u, u_end;   // swapped: unit range; normal: next tile index, tile count
   int kt;
-  bool swap;
+  bool swap, pair;
 };
 
 __device__ __forceinline__ int64_t unit_begin(int64_t c, int64_t U, int64_t G) { return c * U / G; }
@@ -209,16 +235,17 @@ __device__ __forceinline__ int64_t cta_of_unit(int64_t u, int64_t U, int64_t G) 
   return ((u + 1) * G + U - 1) / U - 1;
 }
 
-__device__ __forceinline__ WorkIter work_begin(const GemmParams& p, bool swap) {
+__device__ __forceinline__ WorkIter work_begin(const GemmParams& p, bool swap, bool pair = false) {
   WorkIter w;
   w.kt = p.kt;
   w.swap = swap;
+  w.pair = pair;
   if (swap) {
     const int64_t U = (int64_t)p.tiles_p * p.kt, G = gridDim.x;
     w.u = unit_begin(blockIdx.x, U, G);
     w.u_end = unit_begin(blockIdx.x + 1, U, G);
   } else {
-    w.u = blockIdx.x;
+    w.u = pair ? blockIdx.x / 2 : blockIdx.x;
     w.u_end = (int64_t)p.tiles_p * p.tiles_q;
   }
   return w;
@@ -237,7 +264,7 @@ __device__ __forceinline__ bool work_next(const GemmParams& p, WorkIter& w, int&
     tile_coords(p, (int)w.u, tp, tq);
     kb = 0;
     ke = w.kt;
-    w.u += gridDim.x;
+    w.u += w.pair ? gridDim.x / 2 : gridDim.x;
   }
   return true;
 }
@@ -279,10 +306,10 @@ __device__ __forceinline__ uint64_t ld_word(const uint64_t* p) {
 // stored with the 128B swizzle the output tensor map uses.
 __device__ __forceinline__ uint32_t swz128(uint32_t r, uint32_t c) { return r * 128 + ((c ^ (r & 7)) << 4); }
 
-template <int BN, bool SWAP, bool OUT_F32, int QX = 0, bool MX = false>
-__global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
+template <int BN, bool SWAP, bool OUT_F32, int QX = 0, bool MX = false, bool PAIR = false>
+__global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX, PAIR>::kThreads, Cfg<BN, SWAP, QX, MX, PAIR>::kMinBlocks)
     nvfp4_gemm_kernel(const __grid_constant__ GemmParams p) {
-  using C = Cfg<BN, SWAP, QX, MX>;
+  using C = Cfg<BN, SWAP, QX, MX, PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -301,6 +328,9 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // CTA pairs: rank in the pair; the even CTA (leader) issues the tcgen05 work
+  const uint32_t prank = PAIR ? (cluster_ctarank() & 1u) : 0u;
+  const bool leader = prank == 0;
   // the next kernel in the stream may launch now; it waits for this grid's
   // completion before touching anything this grid reads or writes
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -311,7 +341,9 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
       mbar_init(bar_empty + 8 * s, 1);
     }
     mbar_init(bar_acc_full, 1);
-    mbar_init(bar_acc_empty, 128);
+    // CTA pairs: one arrival per epilogue warp of either CTA; otherwise one
+    // per epilogue thread
+    mbar_init(bar_acc_empty, PAIR ? 8 : 128);
     mbar_init(bar_drain, 1);
     for (int s = 0; s < C::kStages; ++s) mbar_init(bar_sf + 8 * s, C::kCopyWarps);
     for (int i = 0; i < C::kCopyWarps; ++i) mbar_init(bar_cp_drain + 8 * i, 1);
@@ -321,18 +353,31 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
     prefetch_tmap(&p.tmap_p);
     prefetch_tmap(&p.tmap_q);
     if (!SWAP && p.tma_store) prefetch_tmap(&p.tmap_out);
+    if (PAIR) {
+      prefetch_tmap(&p.tmap_sfa);
+      prefetch_tmap(&p.tmap_sfb);
+    }
   }
   if (threadIdx.x >= 64 && threadIdx.x < 64 + NVFP4_MAX_SEGMENTS) {
     seg_end_s[threadIdx.x - 64] = p.seg_end[threadIdx.x - 64];
     seg_alpha_s[threadIdx.x - 64] = p.seg_alpha[threadIdx.x - 64];
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      // both CTAs of the pair allocate together (the same columns in each)
+      tmem_alloc_pair(smem_u32(tmem_holder), C::kTmemAlloc);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_holder), C::kTmemAlloc);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // the even CTA's barriers are initialised before the odd CTA of its pair
+  // can arrive on them
+  if constexpr (PAIR) cluster_sync();
   const uint32_t tmem_base = *tmem_holder;
 
   if (warp == 0) {
@@ -347,11 +392,13 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
       const int kc = p.kc, rb_q = p.rb_q;
       uint32_t issued_mask = 0, last_parity = 0;   // for the drain on abort
       bool ok = true;
+      // p0: this CTA's first row of P (CTA pairs: its 128-row half of the
+      // 256-row tile); q0: the tile's first row of Q
       auto for_steps = [&](WorkIter w, int first, int count, auto&& fn) {
         int tp, tq, kb, ke, j = 0;
         while (j < first + count && work_next(p, w, tp, tq, kb, ke))
           for (int k = kb; k < ke && j < first + count; ++k, ++j)
-            if (j >= first) fn(j, tp * kBM, tq * BN, k);
+            if (j >= first) fn(j, PAIR ? tp * 2 * kBM + (int)prank * kBM : tp * kBM, tq * BN, k);
       };
       auto nsfb_of = [&](int q0) {
         int n = 0;
@@ -362,13 +409,31 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
       };
       auto load_p = [&](int stage, int p0, int k) {
         const uint32_t fb = bar_full + 8 * stage;
-        const uint32_t sf_bytes = (uint32_t)min(C::kChunks, kc - C::kChunks * k) * kSfChunk;
+        const int nch = min(C::kChunks, kc - C::kChunks * k);
+        if constexpr (PAIR) {
+          // into this CTA's shared memory, completing on the even CTA's barrier
+          tma_load_2d_pair(sbase + C::kOffA + stage * C::kABytes, &p.tmap_p, k * C::kRowBytes, p0, fb);
+          tma_load_2d_pair(sbase + C::kOffSfa + stage * C::kSfaBytes, &p.tmap_sfa, 0, (p0 >> 7) * kc + C::kChunks * k,
+                           fb);
+          return;
+        }
         tma_load_2d(sbase + C::kOffA + stage * C::kABytes, &p.tmap_p, k * C::kRowBytes, p0, fb);
         bulk_load(sbase + C::kOffSfa + stage * C::kSfaBytes,
-                  p.sf_p + ((size_t)(p0 >> 7) * kc + C::kChunks * k) * kSfChunk, sf_bytes, fb);
+                  p.sf_p + ((size_t)(p0 >> 7) * kc + C::kChunks * k) * kSfChunk, (uint32_t)nch * kSfChunk, fb);
       };
       auto load_q = [&](int stage, int q0, int k) {
         const uint32_t fb = bar_full + 8 * stage;
+        if constexpr (PAIR) {
+          // this CTA's 128-row half of the weight tile, and the scales of all
+          // 256 rows (both CTAs copy them into their own TMEM)
+          tma_load_2d_pair(sbase + C::kOffB + stage * C::kBBytes, &p.tmap_q, k * C::kRowBytes, q0 + (int)prank * kBM,
+                           fb);
+#pragma unroll
+          for (int rb = 0; rb < 2; ++rb)
+            tma_load_2d_pair(sbase + C::kOffSfb + stage * C::kSfbBytes + rb * C::kChunks * kSfChunk, &p.tmap_sfb, 0,
+                             ((q0 >> 7) + rb) * kc + C::kChunks * k, fb);
+          return;
+        }
         const uint32_t sf_bytes = (uint32_t)min(C::kChunks, kc - C::kChunks * k) * kSfChunk;
         const int nsfb = nsfb_of(q0);
         tma_load_2d(sbase + C::kOffB + stage * C::kBBytes, &p.tmap_q, k * C::kRowBytes, q0, fb);
@@ -379,11 +444,20 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
                       p.sf_q + ((size_t)((q0 >> 7) + rb) * kc + C::kChunks * k) * kSfChunk, sf_bytes, fb);
       };
       auto expect = [&](int stage, int q0, int k) {
-        const uint32_t sf_bytes = (uint32_t)min(C::kChunks, kc - C::kChunks * k) * kSfChunk;
+        if constexpr (PAIR) {
+          // the even CTA's barrier counts both CTAs' bytes (every box moves
+          // its full size; rows past the tensor are zero-filled)
+          if (leader)
+            mbar_arrive_expect_tx(bar_full + 8 * stage,
+                                  2 * (C::kABytes + C::kBBytes + C::kSfaBytes + C::kSfbBytes));
+          return;
+        }
+        const int nch = min(C::kChunks, kc - C::kChunks * k);
+        const uint32_t sf_bytes = (uint32_t)nch * kSfChunk;
         mbar_arrive_expect_tx(bar_full + 8 * stage,
                               C::kABytes + C::kBBytes + sf_bytes * (1 + (C::kQx ? 0 : nsfb_of(q0))));
       };
-      const WorkIter w0 = work_begin(p, SWAP);
+      const WorkIter w0 = work_begin(p, SWAP, PAIR);
       // prologue: the first kStages stages are free
       int npro = 0;
       const bool w_static = p.w_static != 0;
@@ -401,11 +475,21 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
             tma_prefetch_l2_2d(&p.tmap_p, k * C::kRowBytes, p0);
             bulk_prefetch_l2(p.sf_p + ((size_t)(p0 >> 7) * kc + C::kChunks * k) * kSfChunk, sf_bytes);
           } else {
-            tma_prefetch_l2_2d(&p.tmap_q, k * C::kRowBytes, q0);
+            tma_prefetch_l2_2d(&p.tmap_q, k * C::kRowBytes, PAIR ? q0 + (int)prank * kBM : q0);
           }
         }
         npro = j + 1;
       });
+      if (SWAP) {
+        // decode tiles stream each weight byte once: bring the rest of this
+        // CTA's weight range into L2 now, so that HBM keeps streaming while
+        // the preceding kernel finishes (a hint: it reads nothing into the CTA)
+        for_steps(w0, C::kStages, 1 << 30, [&](int, int p0, int, int k) {
+          const uint32_t sf_bytes = (uint32_t)min(C::kChunks, kc - C::kChunks * k) * kSfChunk;
+          tma_prefetch_l2_2d(&p.tmap_p, k * C::kRowBytes, p0);
+          bulk_prefetch_l2(p.sf_p + ((size_t)(p0 >> 7) * kc + C::kChunks * k) * kSfChunk, sf_bytes);
+        });
+      }
       asm volatile("griddepcontrol.wait;" ::: "memory");
       for_steps(w0, 0, npro, [&](int j, int p0, int q0, int k) {
         if (w_static) {
@@ -434,32 +518,37 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         });
       }
-      if (*abort_flag) {
-        // let every issued copy land before the CTA exits
-        for (int s = 0; s < C::kStages; ++s)
-          if (issued_mask & (1u << s)) {
-            volatile int never = 0;
-            (void)mbar_wait(bar_full + 8 * s, (last_parity >> s) & 1, &never, p.err, p.timeout_ns);
-          }
-      }
+      // let every issued copy land before the CTA exits, whichever role may
+      // have given up (when nothing did, the last load of each stage has
+      // already landed and each wait returns at once).  The odd CTA of a
+      // pair cannot see its loads complete (they count on the even CTA's
+      // barrier): it waits until the MMAs have consumed each stage instead,
+      // and the cluster-wide barrier before exit keeps it until the even CTA
+      // has drained.
+      for (int s = 0; s < C::kStages; ++s)
+        if (issued_mask & (1u << s)) {
+          volatile int never = 0;
+          if (leader) (void)mbar_wait(bar_full + 8 * s, (last_parity >> s) & 1, &never, p.err, p.drain_ns);
+          else (void)mbar_wait(bar_empty + 8 * s, (last_parity >> s) & 1, &never, p.err, p.drain_ns);
+        }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     // The whole warp follows the pipeline; lane 0 issues every MMA.  The copy
     // warps waited for each stage's data and moved its scales into TMEM.
-    constexpr uint32_t idesc = MX ? idesc_mxf4(kBM, BN) : idesc_nvf4(kBM, BN);
+    constexpr uint32_t idesc = MX ? idesc_mxf4(C::kMmaM, BN) : idesc_nvf4(C::kMmaM, BN);
     // Descriptors of stage 0, k-block 0; later stages and k-blocks only move
     // the 14-bit start-address field (address >> 4), which never carries.
     const uint64_t a_desc0 = smem_desc(sbase + C::kOffA, 16, C::kSbo, C::kSwizzleLayout);
     const uint64_t b_desc0 = smem_desc(sbase + (C::kQx ? C::kOffAct : C::kOffB), 16, C::kSbo, C::kSwizzleLayout);
     const uint32_t sf_t0 = tmem_base + C::kSfBase;
-    const int kc = p.kc;
     int stage = 0, region = 0, lstep = 0;    // lstep: steps of this CTA so far
     uint32_t phase = 0, acc_phase = 0, acc_buf = 0;
     bool ok = true;
-    WorkIter w = work_begin(p, SWAP);
+    WorkIter w = work_begin(p, SWAP, PAIR);
     int tp, tq, kb0, ke0;
-    while (ok && work_next(p, w, tp, tq, kb0, ke0)) {
+    // CTA pairs: only the even CTA issues (for both)
+    while (ok && leader && work_next(p, w, tp, tq, kb0, ke0)) {
       if (!mbar_wait(bar_acc_empty, acc_phase ^ 1, abort_flag, p.err, p.timeout_ns)) break;
       tc_fence_after();
       const uint32_t acc = tmem_base + (acc_buf ? C::kAcc1Col : 0);
@@ -485,9 +574,14 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
           auto mma = [&](int kb) {
             const int c = MX ? kb >> 1 : kb;
             const uint32_t id = MX ? (uint32_t)(kb & 1) * 2u : 0u;
-            tc_mma_block_scaled<MX>(acc, ad + (uint64_t)(kb * 2), bd + (uint64_t)(kb * 2),
-                                    idesc | (id << 29) | (id << 4), sfa_t + c * 4, sfb_t + c * 4 * C::kSfbBlocks,
-                                    (acc_in | kb) != 0 ? 1u : 0u);
+            if constexpr (PAIR)
+              tc_mma_block_scaled_pair<MX>(acc, ad + (uint64_t)(kb * 2), bd + (uint64_t)(kb * 2),
+                                           idesc | (id << 29) | (id << 4), sfa_t + c * 4,
+                                           sfb_t + c * 4 * C::kSfbBlocks, (acc_in | kb) != 0 ? 1u : 0u);
+            else
+              tc_mma_block_scaled<MX>(acc, ad + (uint64_t)(kb * 2), bd + (uint64_t)(kb * 2),
+                                      idesc | (id << 29) | (id << 4), sfa_t + c * 4, sfb_t + c * 4 * C::kSfbBlocks,
+                                      (acc_in | kb) != 0 ? 1u : 0u);
           };
           if (nkb == C::kKB) {
 #pragma unroll
@@ -495,7 +589,9 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
           } else {
             for (int kb = 0; kb < nkb; ++kb) mma(kb);
           }
-          tc_commit(bar_empty + 8 * stage);
+          // the stage is free in both CTAs of a pair
+          if constexpr (PAIR) tc_commit_pair_both(bar_empty + 8 * stage);
+          else tc_commit(bar_empty + 8 * stage);
         }
         __syncwarp();
         if (++stage == C::kStages) { stage = 0; phase ^= 1; }
@@ -503,17 +599,21 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
         ++lstep;
       }
       if (!ok) break;
-      if (lane == 0) tc_commit(bar_acc_full);
+      if (lane == 0) {
+        if constexpr (PAIR) tc_commit_pair_both(bar_acc_full);
+        else tc_commit(bar_acc_full);
+      }
       __syncwarp();
       acc_phase ^= 1;
       acc_buf ^= 1;
     }
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       // every MMA and scale copy issued by this thread has completed once
       // this commit arrives
-      tc_commit(bar_drain);
+      if constexpr (PAIR) tc_commit_pair(bar_drain);
+      else tc_commit(bar_drain);
       volatile int never = 0;
-      (void)mbar_wait(bar_drain, 0, &never, p.err, p.timeout_ns);
+      (void)mbar_wait(bar_drain, 0, &never, p.err, p.drain_ns);
     }
     __syncwarp();
   } else if (warp < 6) {
@@ -527,7 +627,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
     const bool tma_store = !SWAP && p.tma_store;
     uint32_t acc_phase = 0, acc_buf = 0;
     uint32_t out_buf = 0;                    // next staging buffer (TMA store path)
-    WorkIter w = work_begin(p, SWAP);
+    WorkIter w = work_begin(p, SWAP, PAIR);
     const int64_t U = (int64_t)p.tiles_p * p.kt, G = gridDim.x;
     int tp, tq, kb0, ke0;
     bool first_item = true;
@@ -545,7 +645,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
       int ks[C::kActSteps];
       int nsteps = 0;
       {
-        WorkIter wq = work_begin(p, SWAP);
+        WorkIter wq = work_begin(p, SWAP, PAIR);
         int a, b2, c0, c1;
         while (work_next(p, wq, a, b2, c0, c1))
           for (int k = c0; k < c1 && nsteps < C::kActSteps; ++k) ks[nsteps++] = k;
@@ -614,8 +714,24 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
         }
       }
     }
+    // hand the accumulator back to the MMA warp (CTA pairs: to the even
+    // CTA's MMA warp, one arrival per warp of either CTA)
+    auto release_acc = [&]() {
+      tc_fence_before();
+      if constexpr (PAIR) {
+        __syncwarp();
+        if (lane == 0) {
+          if (leader) mbar_arrive(bar_acc_empty);
+          else mbar_arrive_cluster(map_to_rank(bar_acc_empty, 0));
+        }
+      } else {
+        mbar_arrive(bar_acc_empty);
+      }
+    };
     while (work_next(p, w, tp, tq, kb0, ke0)) {
-      const int64_t p0 = (int64_t)tp * kBM, q0 = (int64_t)tq * BN;
+      // CTA pairs: this CTA's rows are its 128-row half of the 256-row tile
+      const int64_t p0 = PAIR ? (int64_t)tp * 2 * kBM + (int64_t)prank * kBM : (int64_t)tp * kBM;
+      const int64_t q0 = (int64_t)tq * BN;
       if (!mbar_wait(bar_acc_full, acc_phase, abort_flag, p.err, p.timeout_ns)) break;
       __syncwarp();
       tc_fence_after();
@@ -637,10 +753,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
             tmem_ld_32x32b_x32(tacc + col, r0);
             tmem_ld_32x32b_x32(tacc + col + 32, r1);
             tmem_ld_wait();
-            if (slot == C::kSharedSlots - 1 && C::kOverlapAcc) {
-              tc_fence_before();
-              mbar_arrive(bar_acc_empty);
-            }
+            if (slot == C::kSharedSlots - 1 && C::kOverlapAcc) release_acc();
             const int64_t n0 = q0 + col;
             // one scale for the whole 64-column slot unless a segment
             // boundary falls inside it
@@ -674,10 +787,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
               }
             }
           }
-          if (!C::kOverlapAcc) {
-            tc_fence_before();
-            mbar_arrive(bar_acc_empty);
-          }
+          if (!C::kOverlapAcc) release_acc();
           if (tma_store) {
             // 64-column sub-tiles through two 16 KB swizzled staging buffers
 #pragma unroll
@@ -726,10 +836,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
             __syncwarp();
             tmem_ld_32x32b_x32(tacc + c * 32, r);
             tmem_ld_wait();
-            if (cc == 2 * C::kSharedSlots - 1 && C::kOverlapAcc) {
-              tc_fence_before();
-              mbar_arrive(bar_acc_empty);
-            }
+            if (cc == 2 * C::kSharedSlots - 1 && C::kOverlapAcc) release_acc();
             const int64_t n0 = q0 + c * 32;
             int seg_lo = 0, seg_hi = 0;
             if (n_seg > 1) {
@@ -771,10 +878,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
               }
             }
           }
-          if (!C::kOverlapAcc) {
-            tc_fence_before();
-            mbar_arrive(bar_acc_empty);
-          }
+          if (!C::kOverlapAcc) release_acc();
         }
       } else {
         // swap: lane = weight row = output column n; accumulator column =
@@ -859,7 +963,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
                     const int mm = cb * 32 + i;
                     v[i] = q0 + mm < M ? ld_word(src + (int64_t)mm * kBM) : (uint64_t)kFullTag << 32;
                   }
-                  uint32_t all = 1;
+                  uint32_t all = p.test_stall ? 0u : 1u;
 #pragma unroll
                   for (int i = 0; i < kCols; ++i) all &= (uint32_t)((v[i] >> 32) == kFullTag);
                   if (all) break;
@@ -903,7 +1007,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
     // rewritten only once the MMAs that read it last have completed.
     const bool copy_p = warp == 6;
     const int rbq = warp - 7;                   // Q block of this warp
-    if (lane == 0) {
+    if (lane == 0 && leader) {                  // CTA pairs: the even CTA copies for both
       const uint64_t desc0 =
           smem_desc(sbase + (copy_p ? C::kOffSfa : (C::kQx ? C::kOffActSf : C::kOffSfb)), 16, 128, 0);
       const uint32_t sf_t0 = tmem_base + C::kSfBase;
@@ -912,7 +1016,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
       int64_t step = 0;                         // pipeline steps issued so far
       uint32_t phase = 0;
       bool ok = true;
-      WorkIter w = work_begin(p, SWAP);
+      WorkIter w = work_begin(p, SWAP, PAIR);
       int tp, tq, kb0, ke0;
       while (ok && work_next(p, w, tp, tq, kb0, ke0)) {
         for (int k = kb0; k < ke0; ++k) {
@@ -936,7 +1040,10 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
           const int nch = min(C::kChunks, kc - C::kChunks * k);
           if (copy_p) {
             const uint64_t d = desc0 + (uint64_t)((stage * C::kSfaBytes) >> 4);
-            if (nch == C::kChunks) {
+            if constexpr (PAIR) {
+              for (int c = 0; c < nch; ++c)
+                tc_cp_32x128b_warpx4_pair(sfa_t + c * 4, d + (uint64_t)(c * (kSfChunk >> 4)));
+            } else if (nch == C::kChunks) {
 #pragma unroll
               for (int c = 0; c < C::kChunks; ++c)
                 tc_cp_32x128b_warpx4(sfa_t + c * 4, d + (uint64_t)(c * (kSfChunk >> 4)));
@@ -946,11 +1053,17 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
           } else {
             const uint64_t d = desc0 + (uint64_t)((C::kQx ? step * C::kActSfBytes : stage * C::kSfbBytes) >> 4);
             const uint32_t sfb_t = sfa_t + C::kSfaCols;
-            for (int c = 0; c < nch; ++c)
-              tc_cp_32x128b_warpx4(sfb_t + c * 4 * C::kSfbBlocks + rbq * 4,
-                                   d + (uint64_t)((rbq * C::kChunks + c) * (kSfChunk >> 4)));
+            for (int c = 0; c < nch; ++c) {
+              if constexpr (PAIR)
+                tc_cp_32x128b_warpx4_pair(sfb_t + c * 4 * C::kSfbBlocks + rbq * 4,
+                                          d + (uint64_t)((rbq * C::kChunks + c) * (kSfChunk >> 4)));
+              else
+                tc_cp_32x128b_warpx4(sfb_t + c * 4 * C::kSfbBlocks + rbq * 4,
+                                     d + (uint64_t)((rbq * C::kChunks + c) * (kSfChunk >> 4)));
+            }
           }
-          tc_commit(bar_sf + 8 * stage);
+          if constexpr (PAIR) tc_commit_pair(bar_sf + 8 * stage);
+          else tc_commit(bar_sf + 8 * stage);
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
           if (++region == C::kSfRegions) region = 0;
           ++step;
@@ -958,19 +1071,25 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX>::kThreads, 1)
       }
       // every copy issued by this thread has landed before TMEM is freed
       const uint32_t db = bar_cp_drain + 8 * (warp - 6);
-      tc_commit(db);
+      if constexpr (PAIR) tc_commit_pair(db);
+      else tc_commit(db);
       volatile int never = 0;
-      (void)mbar_wait(db, 0, &never, p.err, p.timeout_ns);
+      (void)mbar_wait(db, 0, &never, p.err, p.drain_ns);
     }
     __syncwarp();
   }
 
   tc_fence_before();
   __syncthreads();
+  // no CTA of a cluster leaves while another may still write into, or read
+  // from, its shared memory or TMEM (CTA pairs: the even CTA's tensor-core
+  // work on both has drained)
+  if constexpr (PAIR) cluster_sync();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, C::kTmemAlloc);
+    else tmem_dealloc(tmem_base, C::kTmemAlloc);
   }
 }
 
@@ -1011,6 +1130,20 @@ bool make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, in
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Block scales in the tensor-core order viewed as [chunks, 128] 32-bit words
+// (one 512-byte chunk per row), boxes of `chunks` consecutive chunks.
+bool make_sf_map(CUtensorMap* m, const void* base, int64_t rows, int64_t kc, int chunks) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {128, (cuuint64_t)(ceil_div(rows, 128) * kc)};
+  const cuuint64_t strides[1] = {512};
+  const cuuint32_t box[2] = {128, (cuuint32_t)chunks};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Output [M, N] (bf16 or f32), boxes of 128 rows x 128 bytes, 128B swizzle.
 bool make_out_map(CUtensorMap* m, void* base, int64_t M, int64_t N, bool f32) {
   EncodeTiledFn fn = encode_fn();
@@ -1040,54 +1173,78 @@ bool is_static(const void* p, size_t bytes) {
 }
 
 // Swapped (decode) tiles are split over the CTAs along K; partial tiles are
-// exchanged through a workspace the library owns: one per (device, stream),
-// allocated (all words empty) on the first swapped call on that stream, kept
-// until exit.
+// exchanged through a K-split workspace of one stream: either one the caller
+// registered for that stream (nvfp4_set_workspace: caller-owned, never freed
+// here) or, failing that, one the library allocates on the first swapped
+// call on that stream (all words empty) and frees in
+// nvfp4_release_workspaces().  One per stream, because calls on unordered
+// streams may run at the same time and must not share partial words.
 struct Workspace {
   uint64_t* ws = nullptr;
   size_t bytes = 0;
+  bool owned = false;   // allocated (and freed) by the library
 };
 
 std::mutex g_ws_mu;
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws_table;
 
-cudaError_t get_workspace(const DeviceInfo* d, cudaStream_t st, Workspace* out) {
+// Bytes of K-split workspace a swapped GEMM with activation side bn needs.
+size_t workspace_need(const DeviceInfo* d, int bn) {
+  return (size_t)2 * d->sm_count * (size_t)bn * kBM * sizeof(uint64_t);
+}
+
+cudaError_t get_workspace(const DeviceInfo* d, cudaStream_t st, int bn, Workspace* out) {
   std::lock_guard<std::mutex> lock(g_ws_mu);
   auto it = g_ws_table.find({d->device, st});
   if (it != g_ws_table.end()) {
+    if (it->second.bytes < workspace_need(d, bn)) return cudaErrorInvalidValue;   // a registered one too small
     *out = it->second;
     return cudaSuccess;
   }
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
   if (cudaStreamIsCapturing(st, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) return cudaErrorNotPermitted;
   Workspace w;
-  w.bytes = (size_t)2 * d->sm_count * 128 * kBM * sizeof(uint64_t);
+  w.bytes = workspace_need(d, 128);
+  w.owned = true;
   cudaError_t e = cudaMalloc(&w.ws, w.bytes);
   if (e != cudaSuccess) return e;
   e = cudaMemset(w.ws, 0, w.bytes);
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess) {
+    cudaFree(w.ws);
+    return e;
+  }
   g_ws_table[{d->device, st}] = w;
   *out = w;
   return cudaSuccess;
 }
 
-template <int BN, bool SWAP, bool OUT_F32, int QX = 0, bool MX = false>
-cudaError_t launch(const GemmParams& p, const DeviceInfo* d, cudaStream_t st) {
-  using Cf = Cfg<BN, SWAP, QX, MX>;
-  auto kern = nvfp4_gemm_kernel<BN, SWAP, OUT_F32, QX, MX>;
+template <int BN, bool SWAP, bool OUT_F32, int QX = 0, bool MX = false, bool PAIR = false>
+cudaError_t set_smem_attr(const DeviceInfo* d) {
+  using Cf = Cfg<BN, SWAP, QX, MX, PAIR>;
   static std::once_flag once[64];
   static cudaError_t attr_err[64];
   std::call_once(once[d->device], [&] {
-    attr_err[d->device] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmemBytes);
+    attr_err[d->device] = cudaFuncSetAttribute(nvfp4_gemm_kernel<BN, SWAP, OUT_F32, QX, MX, PAIR>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmemBytes);
   });
-  if (attr_err[d->device] != cudaSuccess) return attr_err[d->device];
-  int grid;
-  if (SWAP) {
-    const int64_t units = (int64_t)p.tiles_p * p.kt;
-    grid = (int)(units < d->sm_count ? units : d->sm_count);
-  } else {
-    const int tiles = p.tiles_p * p.tiles_q;
-    grid = tiles < d->sm_count ? tiles : d->sm_count;
+  return attr_err[d->device];
+}
+
+// grid: number of CTAs (0 = the persistent grid); cluster: CTAs per cluster
+template <int BN, bool SWAP, bool OUT_F32, int QX = 0, bool MX = false, bool PAIR = false>
+cudaError_t launch(const GemmParams& p, const DeviceInfo* d, cudaStream_t st, int grid = 0, int cluster = 1) {
+  using Cf = Cfg<BN, SWAP, QX, MX, PAIR>;
+  auto kern = nvfp4_gemm_kernel<BN, SWAP, OUT_F32, QX, MX, PAIR>;
+  const cudaError_t ea = set_smem_attr<BN, SWAP, OUT_F32, QX, MX, PAIR>(d);
+  if (ea != cudaSuccess) return ea;
+  if (grid == 0) {
+    if (SWAP) {
+      const int64_t units = (int64_t)p.tiles_p * p.kt;
+      grid = (int)(units < d->sm_count ? units : d->sm_count);
+    } else {
+      const int tiles = p.tiles_p * p.tiles_q;
+      grid = tiles < d->sm_count ? tiles : d->sm_count;
+    }
   }
   // programmatic dependent launch: the kernel may start while the previous
   // kernel in the stream finishes; it waits (griddepcontrol.wait) before
@@ -1097,11 +1254,18 @@ cudaError_t launch(const GemmParams& p, const DeviceInfo* d, cudaStream_t st) {
   cfg.blockDim = dim3(Cf::kThreads);
   cfg.dynamicSmemBytes = Cf::kSmemBytes;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (PAIR) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  }
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
@@ -1109,7 +1273,13 @@ float alpha_of(float ga, float gw) { return (float)(1.0 / ((double)ga * (double)
 
 template <bool MX>
 cudaError_t launch_shape(const GemmParams& p, const DeviceInfo* d, cudaStream_t st, bool swap, int bn, bool f32) {
-  if (!swap) return f32 ? launch<256, false, true, 0, MX>(p, d, st) : launch<256, false, false, 0, MX>(p, d, st);
+  if (!swap) {
+    // CTA pairs: 256 x 256 tiles, a persistent grid of whole pairs
+    const int64_t tiles = (int64_t)p.tiles_p * p.tiles_q;
+    const int pairs = (int)(tiles < d->sm_count / 2 ? tiles : d->sm_count / 2);
+    return f32 ? launch<256, false, true, 0, MX, true>(p, d, st, 2 * pairs, 2)
+               : launch<256, false, false, 0, MX, true>(p, d, st, 2 * pairs, 2);
+  }
   if (bn == 16) return f32 ? launch<16, true, true, 0, MX>(p, d, st) : launch<16, true, false, 0, MX>(p, d, st);
   if (bn == 32) return f32 ? launch<32, true, true, 0, MX>(p, d, st) : launch<32, true, false, 0, MX>(p, d, st);
   if (bn == 64) return f32 ? launch<64, true, true, 0, MX>(p, d, st) : launch<64, true, false, 0, MX>(p, d, st);
@@ -1122,7 +1292,7 @@ cudaError_t launch_shape(const GemmParams& p, const DeviceInfo* d, cudaStream_t 
 nvfp4_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float ga, const uint8_t* w_codes,
                       const uint8_t* w_scales, const int64_t* seg_offsets, const float* seg_gs, int n_seg,
                       int64_t M, int64_t N, int64_t K, void* out, nvfp4_out_dtype out_dtype, cudaStream_t st,
-                      bool mx = false) {
+                      bool mx = false, int test_stall = 0) {
   if (!a_codes || !a_scales || !w_codes || !w_scales || !out) return NVFP4_ERR_INVALID_ARG;
   if (M < 1 || N < 1 || K < 32 || K % 32 != 0) return NVFP4_ERR_INVALID_ARG;
   if (M > (1ll << 31) - 256 || N > (1ll << 31) - 256 || K > (1ll << 31)) return NVFP4_ERR_UNSUPPORTED;
@@ -1141,16 +1311,35 @@ nvfp4_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float ga,
 
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
+  const bool f32 = out_dtype == NVFP4_OUT_F32;
+  p.err = d->err_word;
+  p.timeout_ns = wait_timeout_ns();
+  p.drain_ns = drain_timeout_ns();
+  p.M = M;
+  p.N = N;
+  p.n_seg = n_seg;
+  p.test_stall = test_stall;
+  for (int i = 0; i < n_seg; ++i) {
+    p.seg_end[i] = (int)seg_offsets[i + 1];
+    p.seg_alpha[i] = alpha_of(ga, seg_gs[i]);
+  }
+  p.w_static = is_static(w_codes, (size_t)N * (size_t)(K / 2)) &&
+                       is_static(w_scales, nvfp4_scale_bytes(N, mx ? K / 2 : K, NVFP4_SF_TCGEN05))
+                   ? 1 : 0;
+  p.kc = (int)ceil_div(K, mx ? 128 : 64);
+  p.kmma = (int)ceil_div(K, 64);
+  p.out = out;
   const bool swap = M <= 128;
+  int bn = 256;
+  if (swap) bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
   if (swap) {
     Workspace w;
-    const cudaError_t e = get_workspace(d, st, &w);
+    const cudaError_t e = get_workspace(d, st, bn, &w);
     if (e == cudaErrorNotPermitted) return NVFP4_ERR_UNSUPPORTED;
+    if (e == cudaErrorInvalidValue) return NVFP4_ERR_INVALID_ARG;
     if (e != cudaSuccess) return cuda_status(e);
     p.ws = w.ws;
   }
-  int bn = 256;
-  if (swap) bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
   p.rows_p = (int)(swap ? N : M);
   p.rows_q = (int)(swap ? M : N);
   const uint8_t* codes_p = swap ? w_codes : a_codes;
@@ -1158,32 +1347,25 @@ nvfp4_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float ga,
   p.sf_p = swap ? w_scales : a_scales;
   p.sf_q = swap ? a_scales : w_scales;
   const int kkb = swap ? Cfg<16, true>::kKB : Cfg<256, false>::kKB;
+  // normal tiles run as CTA pairs: each CTA loads 128 rows of the 256-row
+  // weight tile, and the scale chunks through tensor maps
   if (!make_code_map(&p.tmap_p, codes_p, p.rows_p, K, kBM, 32 * kkb) ||
-      !make_code_map(&p.tmap_q, codes_q, p.rows_q, K, bn, 32 * kkb))
+      !make_code_map(&p.tmap_q, codes_q, p.rows_q, K, swap ? bn : kBM, 32 * kkb))
     return NVFP4_ERR_CUDA;
-  p.out = out;
-  // TMA stores need 16-byte aligned output rows
-  const bool f32 = out_dtype == NVFP4_OUT_F32;
-  p.tma_store = (!swap && (N * (f32 ? 4 : 2)) % 16 == 0) ? 1 : 0;
-  p.w_static = is_static(w_codes, (size_t)N * (size_t)(K / 2)) &&
-                       is_static(w_scales, nvfp4_scale_bytes(N, mx ? K / 2 : K, NVFP4_SF_TCGEN05))
-                   ? 1 : 0;
-  if (p.tma_store && !make_out_map(&p.tmap_out, out, M, N, f32)) return NVFP4_ERR_CUDA;
-  p.err = d->err_word;
-  p.timeout_ns = wait_timeout_ns();
-  p.M = M;
-  p.N = N;
-  p.rb_q = (int)ceil_div(p.rows_q, 128);
-  p.kc = (int)ceil_div(K, mx ? 128 : 64);
-  p.kmma = (int)ceil_div(K, 64);
-  p.kt = (int)ceil_div(K, 64 * kkb);
-  p.tiles_p = (int)ceil_div(p.rows_p, kBM);
-  p.tiles_q = (int)ceil_div(p.rows_q, bn);
-  p.n_seg = n_seg;
-  for (int i = 0; i < n_seg; ++i) {
-    p.seg_end[i] = (int)seg_offsets[i + 1];
-    p.seg_alpha[i] = alpha_of(ga, seg_gs[i]);
+  if (!swap) {
+    const int chunks = mx ? Cfg<256, false, 0, true>::kChunks : Cfg<256, false>::kChunks;
+    if (!make_sf_map(&p.tmap_sfa, p.sf_p, p.rows_p, p.kc, chunks) ||
+        !make_sf_map(&p.tmap_sfb, p.sf_q, p.rows_q, p.kc, chunks))
+      return NVFP4_ERR_CUDA;
   }
+  // TMA stores need 16-byte aligned output rows
+  p.tma_store = (!swap && (N * (f32 ? 4 : 2)) % 16 == 0) ? 1 : 0;
+  if (p.tma_store && !make_out_map(&p.tmap_out, out, M, N, f32)) return NVFP4_ERR_CUDA;
+  p.rb_q = (int)ceil_div(p.rows_q, 128);
+  p.kt = (int)ceil_div(K, 64 * kkb);
+  p.tiles_p = (int)ceil_div(p.rows_p, swap ? kBM : 2 * kBM);
+  p.tiles_q = (int)ceil_div(p.rows_q, bn);
+  p.group_p = swap ? kGroupP : kGroupP / 2;
   return cuda_status(mx ? launch_shape<true>(p, d, st, swap, bn, f32) : launch_shape<false>(p, d, st, swap, bn, f32));
 }
 
@@ -1210,12 +1392,33 @@ constexpr size_t kNoAllocScratchBytes = (size_t)2 * kNoAllocMaxCtas * kNoAllocMa
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
+// The array's device address on each device, resolved on the first call on
+// that device with it current.  Only a successful lookup is kept, so a lookup
+// that failed (for example a lazy module load under memory pressure) is tried
+// again on the next call.  The address is published with release order and
+// read with acquire order (clear_gemm_scratch reads it from any thread).
 struct NoAllocScratch {
-  std::once_flag once;
-  cudaError_t err = cudaSuccess;
-  uint8_t* ptr = nullptr;
+  std::mutex mu;
+  std::atomic<uint8_t*> ptr{nullptr};
 };
 NoAllocScratch g_noalloc[64];
+
+uint8_t* noalloc_scratch_ptr(int device) {
+  NoAllocScratch& sc = g_noalloc[device];
+  uint8_t* p = sc.ptr.load(std::memory_order_acquire);
+  if (p) return p;
+  std::lock_guard<std::mutex> lock(sc.mu);
+  p = sc.ptr.load(std::memory_order_relaxed);
+  if (p) return p;
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || !addr) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  p = static_cast<uint8_t*>(addr);
+  sc.ptr.store(p, std::memory_order_release);
+  return p;
+}
 
 // Quantize X then multiply.  Given activation buffers, the quantize kernel
 // writes (a_codes, a_scales) and the GEMM reads them.  Without them,
@@ -1259,12 +1462,13 @@ nvfp4_status run_linear(const void* x, nvfp4_in_dtype x_dtype, int64_t M, int64_
   }
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
+  const int bn = M <= 16 ? 16 : 32;
   Workspace w;
-  const cudaError_t e0 = get_workspace(d, st, &w);
+  const cudaError_t e0 = get_workspace(d, st, bn, &w);
   if (e0 == cudaErrorNotPermitted) return NVFP4_ERR_UNSUPPORTED;
+  if (e0 == cudaErrorInvalidValue) return NVFP4_ERR_INVALID_ARG;
   if (e0 != cudaSuccess) return cuda_status(e0);
   p.ws = w.ws;
-  const int bn = M <= 16 ? 16 : 32;
   constexpr int kkb = Cfg<16, true>::kKB;
   p.rows_p = (int)N;
   p.rows_q = (int)M;
@@ -1279,6 +1483,7 @@ nvfp4_status run_linear(const void* x, nvfp4_in_dtype x_dtype, int64_t M, int64_
   p.tma_store = 0;
   p.err = d->err_word;
   p.timeout_ns = wait_timeout_ns();
+  p.drain_ns = drain_timeout_ns();
   p.M = M;
   p.N = N;
   p.rb_q = 1;
@@ -1316,8 +1521,9 @@ cudaError_t clear_gemm_scratch(int device) {
         if (first == cudaSuccess) first = e;
       }
   }
-  if (device >= 0 && device < 64 && g_noalloc[device].ptr) {
-    const cudaError_t e = cudaMemset(g_noalloc[device].ptr, 0, kNoAllocScratchBytes);
+  uint8_t* na = device >= 0 && device < 64 ? g_noalloc[device].ptr.load(std::memory_order_acquire) : nullptr;
+  if (na) {
+    const cudaError_t e = cudaMemset(na, 0, kNoAllocScratchBytes);
     if (first == cudaSuccess) first = e;
   }
   const cudaError_t e = cudaDeviceSynchronize();
@@ -1328,7 +1534,7 @@ namespace {
 
 nvfp4_status run_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_scales, float ga, const uint8_t* w_codes,
                               const uint8_t* w_scales, float gw, int64_t M, int64_t N, int64_t K, void* out,
-                              nvfp4_out_dtype out_dtype, cudaStream_t st) {
+                              nvfp4_out_dtype out_dtype, cudaStream_t st, int test_stall = 0) {
   if (!a_codes || !a_scales || !w_codes || !w_scales || !out) return NVFP4_ERR_INVALID_ARG;
   if (M < 1 || N < 1 || K < 32 || K % 32 != 0) return NVFP4_ERR_INVALID_ARG;
   if (out_dtype != NVFP4_OUT_BF16 && out_dtype != NVFP4_OUT_F32) return NVFP4_ERR_INVALID_ARG;
@@ -1340,16 +1546,15 @@ nvfp4_status run_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_scales, f
   const DeviceInfo* d = device_info();
   if (!d) return NVFP4_ERR_CUDA;
   if (d->major != 10 || d->sm_count > kNoAllocMaxCtas || d->device >= 64) return NVFP4_ERR_UNSUPPORTED;
-  // once per device, with that device current (device_info() reads the
-  // current device): the scratch array's address on it
-  NoAllocScratch& sc = g_noalloc[d->device];
-  std::call_once(sc.once, [&] { sc.err = cudaGetSymbolAddress((void**)&sc.ptr, g_noalloc_scratch); });
-  if (sc.err != cudaSuccess || !sc.ptr) return NVFP4_ERR_CUDA;
+  // with this device current (device_info() reads the current device): the
+  // scratch array's address on it, looked up once and then cached
+  uint8_t* scratch = noalloc_scratch_ptr(d->device);
+  if (!scratch) return NVFP4_ERR_CUDA;
 
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
   const int bn = M <= 16 ? 16 : 32;
-  p.ws = reinterpret_cast<uint64_t*>(sc.ptr);
+  p.ws = reinterpret_cast<uint64_t*>(scratch);
   p.rows_p = (int)N;
   p.rows_q = (int)M;
   p.sf_p = w_scales;
@@ -1362,6 +1567,7 @@ nvfp4_status run_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_scales, f
   p.tma_store = 0;
   p.err = d->err_word;
   p.timeout_ns = wait_timeout_ns();
+  p.drain_ns = drain_timeout_ns();
   p.M = M;
   p.N = N;
   p.rb_q = (int)ceil_div(p.rows_q, 128);
@@ -1371,6 +1577,7 @@ nvfp4_status run_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_scales, f
   p.tiles_p = (int)ceil_div(p.rows_p, kBM);
   p.tiles_q = 1;
   p.n_seg = 1;
+  p.test_stall = test_stall;
   p.seg_end[0] = (int)N;
   p.seg_alpha[0] = alpha_of(ga, gw);
   cudaError_t e;
@@ -1394,6 +1601,57 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float a
   const float gs[1] = {w_global_scale};
   return run_gemm(a_codes, a_scales, a_global_scale, w_codes, w_scales, offs, gs, 1, M, N, K, out, out_dtype,
                   (cudaStream_t)stream);
+}
+
+size_t nvfp4_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || N < 1 || K < 32 || K % 32 != 0) return 0;
+  if (M > 128) return 0;                              // normal tiles do not split K
+  const DeviceInfo* d = device_info();
+  if (!d) return 0;
+  const int bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+  return workspace_need(d, bn);
+}
+
+nvfp4_status nvfp4_set_workspace(nvfp4_stream_t stream, void* workspace, size_t bytes) {
+  const DeviceInfo* d = device_info();
+  if (!d) return NVFP4_ERR_CUDA;
+  const cudaStream_t st = (cudaStream_t)stream;
+  std::lock_guard<std::mutex> lock(g_ws_mu);
+  auto it = g_ws_table.find({d->device, st});
+  if (it != g_ws_table.end() && it->second.owned) {
+    // a workspace the library allocated earlier for this stream: freed once
+    // the device is idle
+    if (cudaDeviceSynchronize() != cudaSuccess) return cuda_status(cudaGetLastError());
+    cudaFree(it->second.ws);
+    g_ws_table.erase(it);
+  } else if (it != g_ws_table.end()) {
+    g_ws_table.erase(it);
+  }
+  if (!workspace) return bytes == 0 ? NVFP4_OK : NVFP4_ERR_INVALID_ARG;   // unregistered
+  if (!aligned16(workspace)) return NVFP4_ERR_ALIGNMENT;
+  if (bytes < workspace_need(d, 16)) return NVFP4_ERR_INVALID_ARG;
+  Workspace w;
+  w.ws = static_cast<uint64_t*>(workspace);
+  w.bytes = bytes;
+  w.owned = false;
+  g_ws_table[{d->device, st}] = w;
+  return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_release_workspaces(void) {
+  const DeviceInfo* d = device_info();
+  if (!d) return NVFP4_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return cuda_status(cudaGetLastError());
+  std::lock_guard<std::mutex> lock(g_ws_mu);
+  for (auto it = g_ws_table.begin(); it != g_ws_table.end();) {
+    if (it->first.first == d->device && it->second.owned) {
+      cudaFree(it->second.ws);
+      it = g_ws_table.erase(it);
+    } else {
+      ++it;
+    }
+  }
+  return NVFP4_OK;
 }
 
 nvfp4_status nvfp4_declare_static(const void* base, size_t bytes) {
@@ -1439,6 +1697,20 @@ nvfp4_status nvfp4_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_scales,
                                 int64_t N, int64_t K, void* out, nvfp4_out_dtype out_dtype, nvfp4_stream_t stream) {
   return run_gemm_noalloc(a_codes, a_scales, a_global_scale, w_codes, w_scales, w_global_scale, M, N, K, out,
                           out_dtype, (cudaStream_t)stream);
+}
+
+nvfp4_status nvfp4_test_gemm_stalled_reduction(const uint8_t* a_codes, const uint8_t* a_scales, float a_global_scale,
+                                               const uint8_t* w_codes, const uint8_t* w_scales, float w_global_scale,
+                                               int64_t M, int64_t N, int64_t K, void* out, nvfp4_out_dtype out_dtype,
+                                               int noalloc, nvfp4_stream_t stream) {
+  if (M > 128) return NVFP4_ERR_UNSUPPORTED;                 // only decode tiles split K
+  if (noalloc)
+    return run_gemm_noalloc(a_codes, a_scales, a_global_scale, w_codes, w_scales, w_global_scale, M, N, K, out,
+                            out_dtype, (cudaStream_t)stream, /*test_stall=*/1);
+  const int64_t offs[2] = {0, N};
+  const float gs[1] = {w_global_scale};
+  return run_gemm(a_codes, a_scales, a_global_scale, w_codes, w_scales, offs, gs, 1, M, N, K, out, out_dtype,
+                  (cudaStream_t)stream, /*mx=*/false, /*test_stall=*/1);
 }
 
 }  // extern "C"

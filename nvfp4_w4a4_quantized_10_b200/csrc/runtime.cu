@@ -20,6 +20,7 @@ DeviceInfo g_info[kMaxDevices];
 std::once_flag g_once[kMaxDevices];
 std::atomic<uint64_t> g_timeout_ns{0};
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s
+constexpr uint64_t kMinDrainNs = 1000000000ull;        // 1 s
 
 void init_device(int dev) {
   DeviceInfo& d = g_info[dev];
@@ -53,6 +54,11 @@ const DeviceInfo* device_info() {
 uint64_t wait_timeout_ns() {
   const uint64_t t = g_timeout_ns.load(std::memory_order_relaxed);
   return t ? t : kDefaultTimeoutNs;
+}
+
+uint64_t drain_timeout_ns() {
+  const uint64_t t = wait_timeout_ns();
+  return t > kMinDrainNs ? t : kMinDrainNs;
 }
 
 // One CTA waits on an mbarrier that nothing arrives on.  The bounded wait

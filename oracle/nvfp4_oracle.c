@@ -22,8 +22,9 @@
  *     [anthology record LIT-800, "Standing in the anthology"; cctest.ai
  *     article, "Main findings"; podcast abstract]
  *
- * Readings taken where the pages are silent (each one is a choice, listed in
- * the design notes):
+ * Readings taken where the pages are silent, each one a choice, numbered
+ * R1-R7 here; the same numbers label them wherever the library, its tests and
+ * its documentation refer to them:
  *   R1  E2M1 is the OCP FP4 layout: bit 3 sign, bits 2..1 exponent (bias 1),
  *       bit 0 mantissa; magnitudes {0,0.5,1,1.5,2,3,4,6}.
  *   R2  E4M3 is OCP FP8 E4M3FN: bias 7, largest finite 448, no infinity,

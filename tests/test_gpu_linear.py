@@ -1,9 +1,10 @@
 """nvfp4_linear: quantize the activation and multiply, through the C-ABI.
 
-For decode shapes one kernel quantizes X into shared memory itself; it must
-give bitwise the same output as nvfp4_quantize followed by nvfp4_gemm (same
-per-block arithmetic, same K split, same summation order), and so the same
-oracle agreement.  Other shapes run those two calls."""
+For decode shapes, without activation buffers, one kernel quantizes X into
+shared memory itself; it must give bitwise the same output as
+nvfp4_quantize followed by nvfp4_gemm (same per-block arithmetic, same K
+split, same summation order), and so the same oracle agreement.  With
+activation buffers the call is exactly those two calls."""
 import numpy as np
 import pytest
 import torch
@@ -24,12 +25,13 @@ def _weights(N, K, seed):
             (wc, wsc, gw))
 
 
-def _two_kernels(x, ga, wcd, wsd, gw, N, out_dtype):
+def _two_kernels(x, ga, wcd, wsd, gw, N, out_dtype, noalloc=False):
     M, K = x.shape
     ac, asc = nv.alloc_quantized(M, K, DEV)
     nv.nvfp4_quantize(x, ga, ac, asc)
     out = torch.empty(M, N, dtype=out_dtype, device=DEV)
-    nv.nvfp4_gemm(ac, asc, ga, wcd, wsd, gw, M, N, K, out)
+    gemm = nv.nvfp4_gemm_noalloc if noalloc else nv.nvfp4_gemm
+    gemm(ac, asc, ga, wcd, wsd, gw, M, N, K, out)
     return out
 
 
@@ -50,6 +52,8 @@ def test_linear_one_kernel_equals_quantize_then_gemm(M, N, K, xdt):
         nv.nvfp4_linear(x, ga, wcd, wsd, gw, N, out)          # no activation buffers: one kernel
         torch.cuda.synchronize()
         assert torch.equal(out, ref), (M, N, K, xdt, out_dtype)
+        # and the allocation-free GEMM runs the same K split: bitwise too
+        assert torch.equal(out, _two_kernels(x, ga, wcd, wsd, gw, N, out_dtype, noalloc=True))
     check_device_error_word()
 
 
@@ -99,9 +103,9 @@ def test_linear_chain_reads_the_previous_layers_output():
     w2c, w2s, g2, _ = _weights(N2, N1, seed=22)
     x = synth.student_t_outliers(M, K1, seed=4, dtype=torch.float32).to(torch.bfloat16).to(DEV)
     ga1 = 2688.0 / float(x.float().abs().max())
-    h_ref = _two_kernels(x, ga1, w1c, w1s, g1, N1, torch.bfloat16)
+    h_ref = _two_kernels(x, ga1, w1c, w1s, g1, N1, torch.bfloat16, noalloc=True)
     ga2 = 2688.0 / float(h_ref.float().abs().max())
-    y_ref = _two_kernels(h_ref, ga2, w2c, w2s, g2, N2, torch.float32)
+    y_ref = _two_kernels(h_ref, ga2, w2c, w2s, g2, N2, torch.float32, noalloc=True)
     torch.cuda.synchronize()
     for _ in range(3):
         h = torch.empty(M, N1, dtype=torch.bfloat16, device=DEV)
@@ -129,6 +133,14 @@ def test_linear_host_equals_the_device_call(M, N, K, buffers, pinned):
     nv.nvfp4_linear_host(x_host, ga, wcd, wsd, gw, N, out_host, x_dev, out_dev, ac, asc)
     torch.cuda.synchronize()
     check_device_error_word()
-    want = _two_kernels(x.to(DEV), ga, wcd, wsd, gw, N, torch.bfloat16)
+    # the same layer called on device buffers: with activation buffers it is
+    # quantize + GEMM, without them the one-kernel form
+    want = torch.empty(M, N, dtype=torch.bfloat16, device=DEV)
+    xd = x.to(DEV)
+    if buffers:
+        ac2, asc2 = nv.alloc_quantized(M, K, DEV)
+        nv.nvfp4_linear(xd, ga, wcd, wsd, gw, N, want, ac2, asc2)
+    else:
+        nv.nvfp4_linear(xd, ga, wcd, wsd, gw, N, want)
     torch.cuda.synchronize()
     assert torch.equal(out_host, want.cpu())

@@ -128,28 +128,24 @@ def test_nvfp4_error_below_mxfp4_on_outlier_activations():
 
 
 def test_mx_prefill_full_size_sampled_rows():
-    # the full MXFP4 prefill launch the benchmark times (32768 x 17408 x 5120);
-    # the oracle computes 24 evenly spread rows
+    # the full MXFP4 prefill launch the benchmark times (32768 x 17408 x 5120)
+    # in FP32 output mode, compared with the oracle at the stated tolerance on
+    # 24 evenly spread rows; the BF16 launch is bitwise its BF16 rounding
     w = synth.PREFILL
     x = synth.activation(w, device=DEV)
     wt = synth.weight(w, device=DEV)
     a_c, a_s = _gpu_mx(x)
     w_c, w_s = _gpu_mx(wt)
-    out = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=DEV)
-    nv.nvfp4_mx_gemm(a_c, a_s, w_c, w_s, w.M, w.N, w.K, out)
+    out32 = torch.empty(w.M, w.N, dtype=torch.float32, device=DEV)
+    nv.nvfp4_mx_gemm(a_c, a_s, w_c, w_s, w.M, w.N, w.K, out32)
+    out16 = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=DEV)
+    nv.nvfp4_mx_gemm(a_c, a_s, w_c, w_s, w.M, w.N, w.K, out16)
     torch.cuda.synchronize()
     check_device_error_word()
+    assert torch.equal(out16, out32.to(torch.bfloat16))
+    del out16
     rows = synth.sample_rows(w.M, 24)
     ac, asc = oracle.mx_quantize(x[rows].float().cpu().numpy())
     wc, wsc = oracle.mx_quantize(wt.float().cpu().numpy())
     ref = oracle.mx_gemm(ac, asc, wc, wsc)
-    got = out[rows].float().cpu().numpy()
-    # bf16 output: one bf16 rounding (<= 2^-9 relative) on top of the fp32 tolerance
-    err = np.abs(got - ref)
-    assert np.all(err <= 2.0 ** -8 * np.abs(ref) + 1e-5 * np.abs(ref).max())
-    a_rows = torch.from_numpy(np.ascontiguousarray(ac)).to(DEV)
-    as_rows = torch.from_numpy(oracle.mx_scales_to_tc(asc, w.K)).to(DEV)
-    out32 = torch.empty(len(rows), w.N, dtype=torch.float32, device=DEV)
-    nv.nvfp4_mx_gemm(a_rows, as_rows, w_c, w_s, len(rows), w.N, w.K, out32)
-    torch.cuda.synchronize()
-    assert_gemm_close(out32.cpu().numpy(), ref, "mx prefill rows")
+    assert_gemm_close(out32[rows].cpu().numpy(), ref, "mx prefill rows")
