@@ -176,10 +176,21 @@ NVFP4_API nvfp4_status nvfp4_swizzle_scales(const uint8_t* rowmajor, int64_t row
  * calls on different streams use different workspaces.  Each launch leaves
  * the words it used empty (zero), so a workspace stays ready for the next.
  * M > 128 uses no workspace.
+ * Co-residency: the split-K grid has one CTA per SM of the device
+ * (multiProcessorCount), and the CTA that sums a split tile waits (bounded)
+ * for partials from CTAs with higher indices.  So every CTA of the grid must
+ * be able to run at the same time.  That holds when the call has the whole
+ * GPU.  It does not hold when the process is limited to fewer SMs than the
+ * device reports (an MPS active-thread percentage, a green context, or
+ * another kernel occupying SMs for longer than the wait bound).  Then the
+ * waits run out and the call reports NVFP4_ERR_TIMEOUT through
+ * nvfp4_last_device_error (nothing hangs).  nvfp4_set_decode_cooperative(1)
+ * makes the driver guarantee co-residency: it launches the grid
+ * cooperatively or refuses it (UNSUPPORTED), at about 1.5 us per call.
  * Errors: INVALID_ARG (also: a registered workspace smaller than
  * nvfp4_workspace_bytes for this shape), ALIGNMENT, UNSUPPORTED (device is
  * not sm_100, or a first decode-shaped call during capture with no
- * workspace), CUDA. */
+ * workspace, or a cooperative split-K grid that cannot be co-resident), CUDA. */
 NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float a_global_scale,
                         const uint8_t* w_codes, const uint8_t* w_scales, float w_global_scale,
                         int64_t M, int64_t N, int64_t K, void* out, nvfp4_out_dtype out_dtype,
@@ -399,6 +410,16 @@ NVFP4_API nvfp4_status nvfp4_last_device_error(void);
 /* Bound (nanoseconds) on every wait inside this library's kernels on all
  * later launches from this process; 0 restores the default (2 s). */
 NVFP4_API void nvfp4_set_wait_timeout_ns(uint64_t ns);
+
+/* Launch the split-K (decode, M <= 128) grids of nvfp4_gemm, nvfp4_linear,
+ * nvfp4_gemm_noalloc, nvfp4_fused_proj and nvfp4_mx_gemm as cooperative
+ * grids (enable != 0) from now on, process-wide; 0 (the default) restores
+ * ordinary launches.  A cooperative grid is admitted only if all of its CTAs
+ * can be resident at once, which the split-K reduction needs (see
+ * nvfp4_gemm); a grid that cannot be returns UNSUPPORTED instead of timing
+ * out.  Results are bitwise the same either way.  Costs about 1.5 us per
+ * decode GEMM on B200.  No counterpart in the pages. */
+NVFP4_API void nvfp4_set_decode_cooperative(int enable);
 
 /* Test entry for the failure path: launches one CTA that waits on an
  * mbarrier nothing ever arrives on, bounded by `timeout_ns`.  The kernel

@@ -69,6 +69,8 @@ _lib.nvfp4_convert_e2m1.argtypes = [_vp, _vp, _i64, _vp]
 _lib.nvfp4_last_device_error.argtypes = []
 _lib.nvfp4_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
 _lib.nvfp4_set_wait_timeout_ns.restype = None
+_lib.nvfp4_set_decode_cooperative.argtypes = [ctypes.c_int]
+_lib.nvfp4_set_decode_cooperative.restype = None
 _lib.nvfp4_test_wait_timeout.argtypes = [ctypes.c_uint64, _vp]
 _lib.nvfp4_test_gemm_stalled_reduction.argtypes = [_vp, _vp, _f32, _vp, _vp, _f32, _i64, _i64, _i64, _vp,
                                                    ctypes.c_int, ctypes.c_int, _vp]
@@ -295,6 +297,10 @@ def nvfp4_last_device_error() -> int:
 
 def nvfp4_set_wait_timeout_ns(ns: int) -> None:
     _lib.nvfp4_set_wait_timeout_ns(int(ns))
+
+
+def nvfp4_set_decode_cooperative(enable: bool) -> None:
+    _lib.nvfp4_set_decode_cooperative(1 if enable else 0)
 
 
 def nvfp4_test_wait_timeout(timeout_ns: int, device=None) -> None:

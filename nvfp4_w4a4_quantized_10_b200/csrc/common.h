@@ -32,6 +32,10 @@ uint64_t wait_timeout_ns();
 // wants quick failure reports) never lets a CTA exit under live copies.
 uint64_t drain_timeout_ns();
 
+// Whether split-K (decode) GEMM grids launch as cooperative grids, which the
+// driver admits only when every CTA can be resident at once.
+bool decode_cooperative();
+
 // Empties every K-split scratch buffer of the GEMM on `device` (after a
 // device-side error left partial words behind).  Synchronous.
 cudaError_t clear_gemm_scratch(int device);
@@ -48,6 +52,8 @@ inline bool finite_positive(float g) {
 inline nvfp4_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return NVFP4_OK;
   (void)cudaGetLastError();  // do not leave a sticky launch error for the caller's next check
+  // a cooperative (co-residency guaranteed) grid that cannot be resident at once
+  if (e == cudaErrorCooperativeLaunchTooLarge) return NVFP4_ERR_UNSUPPORTED;
   return NVFP4_ERR_CUDA;
 }
 

@@ -1259,6 +1259,14 @@ cudaError_t launch(const GemmParams& p, const DeviceInfo* d, cudaStream_t st, in
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // split-K tiles: a tile's first CTA waits for partials from later CTAs,
+  // so the grid (at most one CTA per SM) must be resident at once; opted in,
+  // the driver guarantees that or refuses the launch
+  if (SWAP && decode_cooperative()) {
+    attr[1].id = cudaLaunchAttributeCooperative;
+    attr[1].val.cooperative = 1;
+    cfg.numAttrs = 2;
+  }
   if (PAIR) {
     attr[1].id = cudaLaunchAttributeClusterDimension;
     attr[1].val.clusterDim.x = (unsigned)cluster;

@@ -114,7 +114,8 @@ nvfp4_status nvfp4_mx_quantize(const void* x, nvfp4_in_dtype dtype, int64_t M, i
   const int64_t rows = tc ? ceil_div(M, 128) * 128 : M;
   const int64_t nblk_pad = tc ? 4 * kc : K / 32;
   const int64_t total = rows * nblk_pad * 2;
-  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(ceil_div(total, 512), (int64_t)d->sm_count * 4));
+  // one pass over the tensor, two items per thread (as the NVFP4 quantizer)
+  const int blocks = (int)std::max<int64_t>(1, ceil_div(total, 512));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(blocks);
   cfg.blockDim = dim3(256);

@@ -19,6 +19,7 @@ constexpr int kMaxDevices = 64;
 DeviceInfo g_info[kMaxDevices];
 std::once_flag g_once[kMaxDevices];
 std::atomic<uint64_t> g_timeout_ns{0};
+std::atomic<int> g_decode_coop{0};
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s
 constexpr uint64_t kMinDrainNs = 1000000000ull;        // 1 s
 
@@ -50,6 +51,8 @@ const DeviceInfo* device_info() {
   }
   return &g_info[dev];
 }
+
+bool decode_cooperative() { return g_decode_coop.load(std::memory_order_relaxed) != 0; }
 
 uint64_t wait_timeout_ns() {
   const uint64_t t = g_timeout_ns.load(std::memory_order_relaxed);
@@ -103,6 +106,8 @@ nvfp4_status nvfp4_last_device_error(void) {
 }
 
 void nvfp4_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns, std::memory_order_relaxed); }
+
+void nvfp4_set_decode_cooperative(int enable) { g_decode_coop.store(enable ? 1 : 0, std::memory_order_relaxed); }
 
 nvfp4_status nvfp4_test_wait_timeout(uint64_t timeout_ns, nvfp4_stream_t stream) {
   if (timeout_ns == 0 || timeout_ns > 10000000000ull) return NVFP4_ERR_INVALID_ARG;

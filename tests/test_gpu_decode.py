@@ -121,3 +121,75 @@ def test_decode_mxfp4(M, N, K):
     check_device_error_word()
     assert_gemm_close(out32.cpu().numpy(), ref, f"mx {M}x{N}x{K}")
     assert torch.equal(out16, out32.to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("M,N,K", [(8, 12288, 5120), (16, 4097, 1024), (64, 1000, 2048), (128, 3000, 768)])
+def test_decode_cooperative_launch_is_bitwise_equal(M, N, K):
+    # the opt-in co-residency guarantee changes how the grid is launched, not
+    # what it computes: same K split, same summation order
+    (ac, asc, ga), (wc, wsc, gw) = _operands(M, N, K, seed=7 * M + K)
+    a_d, as_d = to_dev_operand(ac, asc, K)
+    w_d, ws_d = to_dev_operand(wc, wsc, K)
+    default = gpu_gemm(a_d, as_d, ga, w_d, ws_d, gw, M, N, K, torch.float32)
+    x = torch.from_numpy(synth.student_t_outliers(M, K, seed=M, dtype=torch.float32).numpy()).to(DEV)
+    lin_default = torch.empty(M, N, dtype=torch.bfloat16, device=DEV)
+    if M <= 32:
+        nv.nvfp4_linear(x, float(ga), w_d, ws_d, float(gw), N, lin_default)
+    torch.cuda.synchronize()
+    nv.nvfp4_set_decode_cooperative(True)
+    try:
+        coop = gpu_gemm(a_d, as_d, ga, w_d, ws_d, gw, M, N, K, torch.float32)
+        if M <= 32:
+            lin = torch.empty_like(lin_default)
+            nv.nvfp4_linear(x, float(ga), w_d, ws_d, float(gw), N, lin)
+            noalloc = torch.empty(M, N, dtype=torch.float32, device=DEV)
+            nv.nvfp4_gemm_noalloc(a_d, as_d, float(ga), w_d, ws_d, float(gw), M, N, K, noalloc)
+        torch.cuda.synchronize()
+    finally:
+        nv.nvfp4_set_decode_cooperative(False)
+    check_device_error_word()
+    assert torch.equal(coop, default)
+    assert_gemm_close(coop.cpu().numpy(), oracle.gemm(ac, asc, ga, wc, wsc, gw), f"cooperative {M}x{N}x{K}")
+    if M <= 32:
+        assert torch.equal(lin, lin_default)
+        assert torch.equal(noalloc, default)
+
+
+@pytest.mark.parametrize("M,N,K", [(8, 12288, 5120), (16, 2048, 4096), (4, 700, 17408)])
+def test_back_to_back_decode_calls_on_one_stream(M, N, K):
+    # Consecutive split-K GEMMs on one stream share its workspace and overlap
+    # under programmatic dependent launch: each must see only its own
+    # partials.  Different weights per call make a partial taken from the
+    # wrong launch visible in the result.
+    (ac, asc, ga), _ = _operands(M, N, K, seed=M + 2 * K)
+    a_d, as_d = to_dev_operand(ac, asc, K)
+    ws = []
+    for i in range(4):
+        wc, wsc, gw = oracle_quantize(synth.normal((N, K), seed=100 + i, std=0.02 * (i + 1)).numpy())
+        ws.append((*to_dev_operand(wc, wsc, K), gw))
+    refs = []
+    for w_d, ws_d, gw in ws:
+        refs.append(gpu_gemm(a_d, as_d, ga, w_d, ws_d, gw, M, N, K, torch.float32))
+        torch.cuda.synchronize()
+    outs = [torch.empty(M, N, dtype=torch.float32, device=DEV) for _ in range(24)]
+    for i, o in enumerate(outs):
+        w_d, ws_d, gw = ws[i % 4]
+        nv.nvfp4_gemm(a_d, as_d, float(ga), w_d, ws_d, float(gw), M, N, K, o)
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    gouts = [torch.empty(M, N, dtype=torch.float32, device=DEV) for _ in range(24)]
+    with torch.cuda.stream(s):                     # this stream's workspace, before the capture
+        nv.nvfp4_gemm(a_d, as_d, float(ga), ws[0][0], ws[0][1], float(ws[0][2]), M, N, K, gouts[0])
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=s):
+        for i, o in enumerate(gouts):
+            w_d, ws_d, gw = ws[i % 4]
+            nv.nvfp4_gemm(a_d, as_d, float(ga), w_d, ws_d, float(gw), M, N, K, o)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    del g
+    check_device_error_word()
+    for i in range(24):
+        assert torch.equal(outs[i], refs[i % 4]), i
+        assert torch.equal(gouts[i], refs[i % 4]), i
