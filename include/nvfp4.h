@@ -421,6 +421,28 @@ NVFP4_API void nvfp4_set_wait_timeout_ns(uint64_t ns);
  * decode GEMM on B200.  No counterpart in the pages. */
 NVFP4_API void nvfp4_set_decode_cooperative(int enable);
 
+/* 1 if this is the bounds-checked debug build (libnvfp4_debug.so, compiled
+ * with NVFP4_BOUNDS_CHECK=1), 0 for the release build.  In the debug build
+ * every global address a kernel computes itself (scale chunks, codes and
+ * scale bytes, output elements, K-split workspace words, in-kernel
+ * activation loads) is checked against its buffer before use; a failed check
+ * records NVFP4_ERR_DEVICE for nvfp4_last_device_error and the access is
+ * skipped (a load is redirected to the buffer's start), with no trap.  TMA
+ * tiles need no check: the hardware clips them to the tensor.  Same entry
+ * points, same results.  No counterpart in the pages. */
+NVFP4_API int nvfp4_bounds_checked(void);
+
+/* Test entry for the debug build's bounds checks: quantizes x (bf16 [M, K],
+ * K % 64 == 0) into codes [M, K/2] and TCGEN05 scales (full-size buffers,
+ * global scale 1) while telling the kernel that the scale buffer ends one
+ * 512-byte chunk early, so the stores to the last chunk fail their check:
+ * nvfp4_last_device_error() then returns NVFP4_ERR_DEVICE.  Those stores'
+ * real addresses lie inside the caller's buffer; nothing outside any buffer
+ * is touched.  Errors: UNSUPPORTED in the release build (no checks compiled),
+ * INVALID_ARG, ALIGNMENT, CUDA. */
+NVFP4_API nvfp4_status nvfp4_test_bounds_check(const void* x, int64_t M, int64_t K, uint8_t* codes,
+                                               uint8_t* block_scales, nvfp4_stream_t stream);
+
 /* Test entry for the failure path: launches one CTA that waits on an
  * mbarrier nothing ever arrives on, bounded by `timeout_ns`.  The kernel
  * records NVFP4_ERR_TIMEOUT in the device error word and exits; the context

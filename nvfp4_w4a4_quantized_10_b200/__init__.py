@@ -8,7 +8,11 @@ CUDA kernels; there is no CPU fallback.  PyTorch supplies device memory and
 streams.
 
 The library is built in-tree by ``python nvfp4_w4a4_quantized_10_b200/build.py``;
-importing this package without it raises ImportError.
+importing this package without it raises ImportError.  With the environment
+variable NVFP4_DEBUG_BOUNDS=1 the package loads the bounds-checked debug build
+(libnvfp4_debug.so) instead: same entry points and results, and a kernel
+address outside its buffer is reported (NVFP4_ERR_DEVICE from
+nvfp4_last_device_error) instead of being accessed.
 """
 from __future__ import annotations
 
@@ -19,11 +23,12 @@ import re
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libnvfp4.so")
+DEBUG_BOUNDS = os.environ.get("NVFP4_DEBUG_BOUNDS", "0") not in ("", "0")
+LIB_PATH = os.path.join(HERE, "libnvfp4_debug.so" if DEBUG_BOUNDS else "libnvfp4.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "nvfp4.h")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libnvfp4.so is not built ({LIB_PATH}); run "
+    raise ImportError(f"{os.path.basename(LIB_PATH)} is not built ({LIB_PATH}); run "
                       "`python nvfp4_w4a4_quantized_10_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -70,6 +75,9 @@ _lib.nvfp4_last_device_error.argtypes = []
 _lib.nvfp4_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
 _lib.nvfp4_set_wait_timeout_ns.restype = None
 _lib.nvfp4_set_decode_cooperative.argtypes = [ctypes.c_int]
+_lib.nvfp4_bounds_checked.argtypes = []
+_lib.nvfp4_bounds_checked.restype = ctypes.c_int
+_lib.nvfp4_test_bounds_check.argtypes = [_vp, _i64, _i64, _vp, _vp, _vp]
 _lib.nvfp4_set_decode_cooperative.restype = None
 _lib.nvfp4_test_wait_timeout.argtypes = [ctypes.c_uint64, _vp]
 _lib.nvfp4_test_gemm_stalled_reduction.argtypes = [_vp, _vp, _f32, _vp, _vp, _f32, _i64, _i64, _i64, _vp,
@@ -297,6 +305,16 @@ def nvfp4_last_device_error() -> int:
 
 def nvfp4_set_wait_timeout_ns(ns: int) -> None:
     _lib.nvfp4_set_wait_timeout_ns(int(ns))
+
+
+def nvfp4_bounds_checked() -> bool:
+    return bool(_lib.nvfp4_bounds_checked())
+
+
+def nvfp4_test_bounds_check(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor) -> None:
+    M, K = x.shape
+    _check("nvfp4_test_bounds_check",
+           _lib.nvfp4_test_bounds_check(_ptr(x), M, K, _ptr(codes), _ptr(scales), _stream(x)))
 
 
 def nvfp4_set_decode_cooperative(enable: bool) -> None:

@@ -91,6 +91,11 @@ struct alignas(64) GemmParams {
   const void* x;
   float x_gs;
   int64_t K;
+  // buffer extents, checked by the debug build's bounds checks
+  uint64_t sf_p_bytes, sf_q_bytes;   // scale buffers
+  uint64_t out_elems;                // M * N
+  uint64_t ws_words;                 // K-split workspace, 64-bit words
+  uint64_t x_bytes;                  // in-kernel activation X
 };
 
 // QX: 0 = the Q operand (activations) arrives quantized, as codes and scales
@@ -418,8 +423,9 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX, PAIR>::kThreads, Cfg<BN,
           return;
         }
         tma_load_2d(sbase + C::kOffA + stage * C::kABytes, &p.tmap_p, k * C::kRowBytes, p0, fb);
-        bulk_load(sbase + C::kOffSfa + stage * C::kSfaBytes,
-                  p.sf_p + ((size_t)(p0 >> 7) * kc + C::kChunks * k) * kSfChunk, (uint32_t)nch * kSfChunk, fb);
+        size_t off = ((size_t)(p0 >> 7) * kc + C::kChunks * k) * kSfChunk;
+        if (!bounds_ok(off + (size_t)nch * kSfChunk <= p.sf_p_bytes, p.err)) off = 0;
+        bulk_load(sbase + C::kOffSfa + stage * C::kSfaBytes, p.sf_p + off, (uint32_t)nch * kSfChunk, fb);
       };
       auto load_q = [&](int stage, int q0, int k) {
         const uint32_t fb = bar_full + 8 * stage;
@@ -439,9 +445,12 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX, PAIR>::kThreads, Cfg<BN,
         tma_load_2d(sbase + C::kOffB + stage * C::kBBytes, &p.tmap_q, k * C::kRowBytes, q0, fb);
 #pragma unroll
         for (int rb = 0; rb < C::kSfbBlocks; ++rb)
-          if (rb < nsfb)
-            bulk_load(sbase + C::kOffSfb + stage * C::kSfbBytes + rb * C::kChunks * kSfChunk,
-                      p.sf_q + ((size_t)((q0 >> 7) + rb) * kc + C::kChunks * k) * kSfChunk, sf_bytes, fb);
+          if (rb < nsfb) {
+            size_t off = ((size_t)((q0 >> 7) + rb) * kc + C::kChunks * k) * kSfChunk;
+            if (!bounds_ok(off + sf_bytes <= p.sf_q_bytes, p.err)) off = 0;
+            bulk_load(sbase + C::kOffSfb + stage * C::kSfbBytes + rb * C::kChunks * kSfChunk, p.sf_q + off, sf_bytes,
+                      fb);
+          }
       };
       auto expect = [&](int stage, int q0, int k) {
         if constexpr (PAIR) {
@@ -473,7 +482,8 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX, PAIR>::kThreads, Cfg<BN,
           const uint32_t sf_bytes = (uint32_t)min(C::kChunks, kc - C::kChunks * k) * kSfChunk;
           if (SWAP) {
             tma_prefetch_l2_2d(&p.tmap_p, k * C::kRowBytes, p0);
-            bulk_prefetch_l2(p.sf_p + ((size_t)(p0 >> 7) * kc + C::kChunks * k) * kSfChunk, sf_bytes);
+            const size_t off = ((size_t)(p0 >> 7) * kc + C::kChunks * k) * kSfChunk;
+            if (bounds_ok(off + sf_bytes <= p.sf_p_bytes, p.err)) bulk_prefetch_l2(p.sf_p + off, sf_bytes);
           } else {
             tma_prefetch_l2_2d(&p.tmap_q, k * C::kRowBytes, PAIR ? q0 + (int)prank * kBM : q0);
           }
@@ -487,7 +497,8 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX, PAIR>::kThreads, Cfg<BN,
         for_steps(w0, C::kStages, 1 << 30, [&](int, int p0, int, int k) {
           const uint32_t sf_bytes = (uint32_t)min(C::kChunks, kc - C::kChunks * k) * kSfChunk;
           tma_prefetch_l2_2d(&p.tmap_p, k * C::kRowBytes, p0);
-          bulk_prefetch_l2(p.sf_p + ((size_t)(p0 >> 7) * kc + C::kChunks * k) * kSfChunk, sf_bytes);
+          const size_t off = ((size_t)(p0 >> 7) * kc + C::kChunks * k) * kSfChunk;
+          if (bounds_ok(off + sf_bytes <= p.sf_p_bytes, p.err)) bulk_prefetch_l2(p.sf_p + off, sf_bytes);
         });
       }
       asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -669,7 +680,12 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX, PAIR>::kThreads, Cfg<BN,
         for (int u = 0; u < kWin; ++u) {
           const int jj = j0 + u;
           const int64_t e = (int64_t)(jj < nsteps ? ks[jj] : 0) * 256 + bq * 16;
-          if (jj < nsteps && e < K) load_block_at<kF32>(xb + ((int64_t)m * K + e) * kEsz, B[u]);
+          if (jj < nsteps && e < K) {
+            if (bounds_ok((uint64_t)((int64_t)m * K + e + 16) * kEsz <= p.x_bytes, p.err))
+              load_block_at<kF32>(xb + ((int64_t)m * K + e) * kEsz, B[u]);
+            else
+              B[u] = Block16<kF32>{};
+          }
         }
       };
       Block16<kF32> Bc[kWin], Bn[kWin];
@@ -822,7 +838,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX, PAIR>::kThreads, Cfg<BN,
               const int64_t n = q0 + slot_col(c / 8) + (c % 8) * 8;
 #pragma unroll
               for (int e = 0; e < 8; ++e)
-                if (n + e < N)
+                if (n + e < N && bounds_ok((uint64_t)(m * N + n + e) < p.out_elems, p.err))
                   reinterpret_cast<uint16_t*>(orow)[n + e] = (uint16_t)(packed[4 * c + e / 2] >> (16 * (e & 1)));
             }
           }
@@ -874,7 +890,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX, PAIR>::kThreads, Cfg<BN,
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
                 const int64_t n = q0 + c * 32 + i;
-                if (n < N) orow[n] = __uint_as_float(r[i]);
+                if (n < N && bounds_ok((uint64_t)(m * N + n) < p.out_elems, p.err)) orow[n] = __uint_as_float(r[i]);
               }
             }
           }
@@ -906,6 +922,7 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX, PAIR>::kThreads, Cfg<BN,
         tc_fence_before();
         mbar_arrive(bar_acc_empty);
         auto store_out = [&](int64_t mm, float v) {
+          if (!bounds_ok((uint64_t)(mm * N + n) < p.out_elems, p.err)) return;
           if constexpr (OUT_F32) reinterpret_cast<float*>(p.out)[mm * N + n] = v;
           else reinterpret_cast<__nv_bfloat16*>(p.out)[mm * N + n] = __float2bfloat16_rn(v);
         };
@@ -934,13 +951,15 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX, PAIR>::kThreads, Cfg<BN,
           // polls each word until it is full and clears it for the next
           // launch.
           if ((int64_t)blockIdx.x != c_first) {
-            uint64_t* part = p.ws + (2 * (int64_t)blockIdx.x + (first_item ? 0 : 1)) * BN * kBM + row;
+            const int64_t part0 = (2 * (int64_t)blockIdx.x + (first_item ? 0 : 1)) * BN * kBM + row;
+            uint64_t* part = p.ws + part0;
 #pragma unroll
             for (int c = 0; c < (BN + 31) / 32; ++c)
 #pragma unroll
               for (int i = 0; i < kCols; ++i) {
                 const int mm = c * 32 + i;
-                if (q0 + mm < M) st_full_word(part + (int64_t)mm * kBM, r[c][i]);
+                if (q0 + mm < M && bounds_ok((uint64_t)(part0 + (int64_t)mm * kBM) < p.ws_words, p.err))
+                  st_full_word(part + (int64_t)mm * kBM, r[c][i]);
               }
           } else {
             float sum[(BN + 31) / 32][kCols];
@@ -951,6 +970,11 @@ __global__ void __launch_bounds__(Cfg<BN, SWAP, QX, MX, PAIR>::kThreads, Cfg<BN,
             bool ok_all = true;
             for (int64_t c = c_first + 1; c <= c_last && ok_all; ++c) {
               const int64_t slot = 2 * c + (unit_begin(c, U, G) >= tile_u0 ? 0 : 1);
+              // the slot's last word is inside the workspace (debug build)
+              if (!bounds_ok((uint64_t)((slot + 1) * BN * kBM) <= p.ws_words, p.err)) {
+                ok_all = false;
+                break;
+              }
               uint64_t* src = p.ws + slot * BN * kBM + row;
               // one round polls every word of a 32-column chunk at once
 #pragma unroll
@@ -1347,6 +1371,7 @@ nvfp4_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float ga,
     if (e == cudaErrorInvalidValue) return NVFP4_ERR_INVALID_ARG;
     if (e != cudaSuccess) return cuda_status(e);
     p.ws = w.ws;
+    p.ws_words = w.bytes / sizeof(uint64_t);
   }
   p.rows_p = (int)(swap ? N : M);
   p.rows_q = (int)(swap ? M : N);
@@ -1370,6 +1395,9 @@ nvfp4_status run_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float ga,
   p.tma_store = (!swap && (N * (f32 ? 4 : 2)) % 16 == 0) ? 1 : 0;
   if (p.tma_store && !make_out_map(&p.tmap_out, out, M, N, f32)) return NVFP4_ERR_CUDA;
   p.rb_q = (int)ceil_div(p.rows_q, 128);
+  p.sf_p_bytes = (uint64_t)ceil_div(p.rows_p, 128) * p.kc * kSfChunk;
+  p.sf_q_bytes = (uint64_t)p.rb_q * p.kc * kSfChunk;
+  p.out_elems = (uint64_t)M * (uint64_t)N;
   p.kt = (int)ceil_div(K, 64 * kkb);
   p.tiles_p = (int)ceil_div(p.rows_p, swap ? kBM : 2 * kBM);
   p.tiles_q = (int)ceil_div(p.rows_q, bn);
@@ -1477,6 +1505,7 @@ nvfp4_status run_linear(const void* x, nvfp4_in_dtype x_dtype, int64_t M, int64_
   if (e0 == cudaErrorInvalidValue) return NVFP4_ERR_INVALID_ARG;
   if (e0 != cudaSuccess) return cuda_status(e0);
   p.ws = w.ws;
+  p.ws_words = w.bytes / sizeof(uint64_t);
   constexpr int kkb = Cfg<16, true>::kKB;
   p.rows_p = (int)N;
   p.rows_q = (int)M;
@@ -1506,6 +1535,9 @@ nvfp4_status run_linear(const void* x, nvfp4_in_dtype x_dtype, int64_t M, int64_
   p.x = x;
   p.x_gs = ga;
   p.K = K;
+  p.sf_p_bytes = (uint64_t)ceil_div(N, 128) * p.kc * kSfChunk;
+  p.out_elems = (uint64_t)M * (uint64_t)N;
+  p.x_bytes = (uint64_t)M * (uint64_t)K * (x_dtype == NVFP4_IN_F32 ? 4 : 2);
   const bool f32 = out_dtype == NVFP4_OUT_F32;
   const bool xf32 = x_dtype == NVFP4_IN_F32;
   cudaError_t e;
@@ -1563,6 +1595,7 @@ nvfp4_status run_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_scales, f
   std::memset(&p, 0, sizeof(p));
   const int bn = M <= 16 ? 16 : 32;
   p.ws = reinterpret_cast<uint64_t*>(scratch);
+  p.ws_words = kNoAllocScratchBytes / sizeof(uint64_t);
   p.rows_p = (int)N;
   p.rows_q = (int)M;
   p.sf_p = w_scales;
@@ -1588,6 +1621,9 @@ nvfp4_status run_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_scales, f
   p.test_stall = test_stall;
   p.seg_end[0] = (int)N;
   p.seg_alpha[0] = alpha_of(ga, gw);
+  p.sf_p_bytes = (uint64_t)ceil_div(N, 128) * p.kc * kSfChunk;
+  p.sf_q_bytes = (uint64_t)p.rb_q * p.kc * kSfChunk;
+  p.out_elems = (uint64_t)M * (uint64_t)N;
   cudaError_t e;
   const bool f32 = out_dtype == NVFP4_OUT_F32;
   if (bn == 16) e = f32 ? launch<16, true, true>(p, d, st) : launch<16, true, false>(p, d, st);

@@ -25,6 +25,7 @@
 
 #include "block_quant.cuh"
 #include "common.h"
+#include "ptx.cuh"
 
 namespace nvfp4 {
 
@@ -37,7 +38,8 @@ template <bool kF32, bool kTC>
 __global__ void __launch_bounds__(256) mx_quantize_kernel(const void* __restrict__ x, int64_t M, int64_t K,
                                                           int64_t nblk_pad, int64_t total_items,
                                                           uint8_t* __restrict__ codes,
-                                                          uint8_t* __restrict__ scales, int64_t kc) {
+                                                          uint8_t* __restrict__ scales, int64_t kc,
+                                                          uint64_t codes_bytes, uint64_t scale_bytes, unsigned* err) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31;
@@ -81,14 +83,15 @@ __global__ void __launch_bounds__(256) mx_quantize_kernel(const void* __restrict
           lo[i] = f[i] * inv;
           hi[i] = f[8 + i] * inv;
         }
-        *reinterpret_cast<uint2*>(codes + r[u] * (K / 2) + j[u] * 16 + h[u] * 8) =
-            make_uint2(cvt_e2m1x8(lo), cvt_e2m1x8(hi));
+        const int64_t co = r[u] * (K / 2) + j[u] * 16 + h[u] * 8;
+        if (bounds_ok((uint64_t)co + 8 <= codes_bytes, err))
+          *reinterpret_cast<uint2*>(codes + co) = make_uint2(cvt_e2m1x8(lo), cvt_e2m1x8(hi));
       }
       if (h[u] == 0) {
         const int64_t off = kTC ? ((r[u] >> 7) * kc + (j[u] >> 2)) * 512 + (r[u] & 31) * 16 + ((r[u] >> 5) & 3) * 4 +
                                       (j[u] & 3)
                                 : r[u] * nblk + j[u];
-        scales[off] = real[u] ? (uint8_t)sbyte : (uint8_t)0;
+        if (bounds_ok((uint64_t)off < scale_bytes, err)) scales[off] = real[u] ? (uint8_t)sbyte : (uint8_t)0;
       }
     }
   }
@@ -126,11 +129,13 @@ nvfp4_status nvfp4_mx_quantize(const void* x, nvfp4_in_dtype dtype, int64_t M, i
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const bool f32 = dtype == NVFP4_IN_F32;
+  const uint64_t codes_bytes = (uint64_t)M * (uint64_t)(K / 2);
+  const uint64_t scale_bytes = tc ? (uint64_t)(rows / 128) * kc * 512 : (uint64_t)M * (uint64_t)(K / 32);
   cudaError_t e;
-  if (f32) e = tc ? cudaLaunchKernelEx(&cfg, mx_quantize_kernel<true, true>, x, M, K, nblk_pad, total, codes, scales, kc)
-                  : cudaLaunchKernelEx(&cfg, mx_quantize_kernel<true, false>, x, M, K, nblk_pad, total, codes, scales, kc);
-  else e = tc ? cudaLaunchKernelEx(&cfg, mx_quantize_kernel<false, true>, x, M, K, nblk_pad, total, codes, scales, kc)
-              : cudaLaunchKernelEx(&cfg, mx_quantize_kernel<false, false>, x, M, K, nblk_pad, total, codes, scales, kc);
+  if (f32) e = tc ? cudaLaunchKernelEx(&cfg, mx_quantize_kernel<true, true>, x, M, K, nblk_pad, total, codes, scales, kc, codes_bytes, scale_bytes, d->err_word)
+                  : cudaLaunchKernelEx(&cfg, mx_quantize_kernel<true, false>, x, M, K, nblk_pad, total, codes, scales, kc, codes_bytes, scale_bytes, d->err_word);
+  else e = tc ? cudaLaunchKernelEx(&cfg, mx_quantize_kernel<false, true>, x, M, K, nblk_pad, total, codes, scales, kc, codes_bytes, scale_bytes, d->err_word)
+              : cudaLaunchKernelEx(&cfg, mx_quantize_kernel<false, false>, x, M, K, nblk_pad, total, codes, scales, kc, codes_bytes, scale_bytes, d->err_word);
   return cuda_status(e);
 }
 

@@ -14,6 +14,30 @@ namespace nvfp4 {
 constexpr unsigned kErrTimeout = 5u;
 constexpr unsigned kErrBounds = 6u;
 
+// Index bounds checks of the debug build (libnvfp4_debug.so, compiled with
+// NVFP4_BOUNDS_CHECK=1).  Every global address a kernel computes itself
+// (not a TMA tile, which the hardware clips) is checked against the size of
+// its buffer before use: a failed check records kErrBounds in the device
+// error word and the caller skips the access (a load is redirected to the
+// buffer's first bytes, so the barrier's byte count still completes).  No
+// trap, no assert.  In the release build the check is compiled out.
+#ifndef NVFP4_BOUNDS_CHECK
+#define NVFP4_BOUNDS_CHECK 0
+#endif
+
+__device__ __forceinline__ bool bounds_ok(bool ok, unsigned* err) {
+#if NVFP4_BOUNDS_CHECK
+  if (!ok) {
+    atomicCAS(err, 0u, kErrBounds);
+    return false;
+  }
+#else
+  (void)ok;
+  (void)err;
+#endif
+  return true;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

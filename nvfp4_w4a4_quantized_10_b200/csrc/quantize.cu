@@ -68,7 +68,8 @@ __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ 
                                                        uint32_t total_blocks, uint32_t nblk, DivU32 div_nblk,
                                                        float g, uint8_t* __restrict__ codes,
                                                        uint8_t* __restrict__ scales, float* amax_out,
-                                                       int64_t kc) {
+                                                       int64_t kc, uint64_t codes_bytes, uint64_t scale_bytes,
+                                                       unsigned* err) {
   constexpr int U = 2;
   // programmatic dependent launch: let the next kernel (the GEMM) start its
   // prologue and weight loads now, and wait until the previous kernel in the
@@ -103,18 +104,23 @@ __global__ void __launch_bounds__(256) quantize_kernel(const void* __restrict__ 
       float amax;
       const uint32_t s = quantize_block<kF32>(B[u], g, rtab, lo, hi, &amax);
       if constexpr (kAmax) local_max = fmaxf(local_max, amax);
-      if (b < real_blocks) reinterpret_cast<uint2*>(codes)[b] = make_uint2(lo, hi);
+      if (b < real_blocks && bounds_ok((uint64_t)(b + 1) * 8 <= codes_bytes, err))
+        reinterpret_cast<uint2*>(codes)[b] = make_uint2(lo, hi);
       if constexpr (kTC) {
         const uint32_t row = div_u32(b, div_nblk);
         const uint32_t j = b - row * nblk;
-        scales[tc_scale_offset(row, j, kc)] = (uint8_t)s;
+        const int64_t o = tc_scale_offset(row, j, kc);
+        if (bounds_ok((uint64_t)o < scale_bytes, err)) scales[o] = (uint8_t)s;
         // K % 64 == 32: the last chunk of the row has two padding slots
         if (j == nblk - 1 && (nblk & 3) == 2) {
-          scales[tc_scale_offset(row, j + 1, kc)] = 0;
-          scales[tc_scale_offset(row, j + 2, kc)] = 0;
+          const int64_t o1 = tc_scale_offset(row, j + 1, kc), o2 = tc_scale_offset(row, j + 2, kc);
+          if (bounds_ok((uint64_t)o1 < scale_bytes && (uint64_t)o2 < scale_bytes, err)) {
+            scales[o1] = 0;
+            scales[o2] = 0;
+          }
         }
       } else {
-        scales[b] = (uint8_t)s;
+        if (bounds_ok((uint64_t)b < scale_bytes, err)) scales[b] = (uint8_t)s;
       }
     }
   }
@@ -255,8 +261,10 @@ cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, float g, uint8_
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  const uint64_t codes_bytes = (uint64_t)M * (uint64_t)(K / 2);
+  const uint64_t scale_bytes = kTC ? (uint64_t)(rows_total / 128) * kc * 512 : (uint64_t)M * (uint64_t)(K / 16);
   return cudaLaunchKernelEx(&cfg, quantize_kernel<kF32, kTC, kAmax>, x, real, total, nblk, make_div(nblk), g, codes,
-                            scales, amax_out, kc);
+                            scales, amax_out, kc, codes_bytes, scale_bytes, d->err_word);
 }
 
 cudaError_t launch_amax(const void* x, bool f32, int64_t n_vec, float* amax_out, cudaStream_t st,
@@ -355,6 +363,29 @@ nvfp4_status nvfp4_quantize(const void* x, nvfp4_in_dtype dtype, int64_t M, int6
   else NVFP4_Q(true, true, false) else NVFP4_Q(true, true, true) else e = cudaErrorInvalidValue;
 #undef NVFP4_Q
   return cuda_status(e);
+}
+
+nvfp4_status nvfp4_test_bounds_check(const void* x, int64_t M, int64_t K, uint8_t* codes, uint8_t* block_scales,
+                                     nvfp4_stream_t stream) {
+  if (!NVFP4_BOUNDS_CHECK) return NVFP4_ERR_UNSUPPORTED;   // the release build has no checks to exercise
+  if (!x || !codes || !block_scales || M < 1 || K < 64 || K % 64 != 0) return NVFP4_ERR_INVALID_ARG;
+  if (ceil_div(M, 128) * 128 * (K / 16) >= (1ll << 31)) return NVFP4_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(block_scales)) return NVFP4_ERR_ALIGNMENT;
+  const DeviceInfo* d = device_info();
+  if (!d) return NVFP4_ERR_CUDA;
+  // the quantizer, told that the scale buffer ends one 512-byte chunk early:
+  // the scales of the last chunk fail the check (their real addresses are
+  // inside the caller's full-size buffer, so nothing out of range is touched)
+  const int64_t rows_total = ceil_div(M, 128) * 128, kc = K / 64;
+  const uint32_t nblk = (uint32_t)(K / 16);
+  const uint32_t real = (uint32_t)(M * (K / 16)), total = (uint32_t)(rows_total * (K / 16));
+  const uint64_t codes_bytes = (uint64_t)M * (uint64_t)(K / 2);
+  const uint64_t short_scales = (uint64_t)(rows_total / 128) * kc * 512 - 512;
+  const int blocks = grid_for(ceil_div(total, 2), 256, d, 1 << 20);
+  quantize_kernel<false, true, false><<<blocks, 256, 0, (cudaStream_t)stream>>>(
+      x, real, total, nblk, make_div(nblk), 1.0f, codes, block_scales, nullptr, kc, codes_bytes, short_scales,
+      d->err_word);
+  return cuda_status(cudaGetLastError());
 }
 
 nvfp4_status nvfp4_swizzle_scales(const uint8_t* rowmajor, int64_t rows, int64_t K, uint8_t* tc,

@@ -107,6 +107,8 @@ nvfp4_status nvfp4_last_device_error(void) {
 
 void nvfp4_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns, std::memory_order_relaxed); }
 
+int nvfp4_bounds_checked(void) { return NVFP4_BOUNDS_CHECK ? 1 : 0; }
+
 void nvfp4_set_decode_cooperative(int enable) { g_decode_coop.store(enable ? 1 : 0, std::memory_order_relaxed); }
 
 nvfp4_status nvfp4_test_wait_timeout(uint64_t timeout_ns, nvfp4_stream_t stream) {

@@ -21,6 +21,19 @@ def test_every_declared_symbol_is_exported():
         assert hasattr(nv, n), n
 
 
+def test_debug_build_exports_the_same_symbols():
+    # the bounds-checked twin (NVFP4_DEBUG_BOUNDS=1) is a drop-in replacement
+    import os
+    path = os.path.join(os.path.dirname(nv.LIB_PATH), "libnvfp4_debug.so")
+    assert os.path.exists(path), path
+    dbg = ctypes.CDLL(path)
+    for n in nv.declared_symbols():
+        assert hasattr(dbg, n), n
+    dbg.nvfp4_bounds_checked.restype = ctypes.c_int
+    assert dbg.nvfp4_bounds_checked() == 1
+    assert nv.nvfp4_bounds_checked() == nv.DEBUG_BOUNDS
+
+
 def test_status_strings_and_version():
     assert nv.version() >= 100
     for s in range(7):
