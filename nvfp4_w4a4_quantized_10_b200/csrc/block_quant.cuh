@@ -16,6 +16,30 @@
 
 namespace nvfp4 {
 
+// Unsigned division by an invariant divisor d (Granlund and Montgomery,
+// "Division by invariant integers using multiplication", 1994, unsigned
+// case): with l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1,
+// n / d == (mulhi(n, m) + n) >> l for every 32-bit n.
+struct DivU32 {
+  uint32_t m, l;
+};
+
+__device__ __forceinline__ uint32_t div_u32(uint32_t n, DivU32 d) {
+  const uint32_t t = __umulhi(n, d.m);
+  return (uint32_t)(((uint64_t)t + n) >> d.l);
+}
+
+// Host side: the (m, l) pair for divisor d >= 1.
+inline DivU32 make_div(uint32_t d) {
+  uint32_t l = 0;
+  while ((1ull << l) < d) ++l;
+  DivU32 r;
+  r.l = l;
+  r.m = (uint32_t)((((1ull << l) - d) << 32) / d + 1);
+  return r;
+}
+
+
 // ----------------------------------------------------------------- encoders
 
 __device__ __forceinline__ uint32_t cvt_e4m3(float t) {

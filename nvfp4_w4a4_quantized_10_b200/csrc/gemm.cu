@@ -137,7 +137,10 @@ struct Cfg {
   static constexpr int kActCodeBytes = BN * kRowBytes;
   static constexpr int kActSfBytes = kKB * kSfChunk;
   static constexpr int kActBytes = kActSteps * (kActCodeBytes + kActSfBytes);
-  static constexpr int kMaxStages = 8;
+  // CTA pairs keep 4 stages although 5 fit: 5 ran 2-7 % slower on every
+  // prefill and fused shape measured (the deeper ring lets the copy warps
+  // run further ahead of MMAs that are not waiting on data)
+  static constexpr int kMaxStages = PAIR ? 4 : 8;
   // Decode tiles with a small activation side run two CTAs per SM: the next
   // GEMM on the stream (programmatic dependent launch) then starts at once
   // beside this one and streams its weight while this one finishes, instead

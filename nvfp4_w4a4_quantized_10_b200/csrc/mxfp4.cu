@@ -36,7 +36,7 @@ namespace nvfp4 {
 // write a zero scale byte.
 template <bool kF32, bool kTC>
 __global__ void __launch_bounds__(256) mx_quantize_kernel(const void* __restrict__ x, int64_t M, int64_t K,
-                                                          int64_t nblk_pad, int64_t total_items,
+                                                          int64_t nblk_pad, DivU32 div_nblk_pad, int64_t total_items,
                                                           uint8_t* __restrict__ codes,
                                                           uint8_t* __restrict__ scales, int64_t kc,
                                                           uint64_t codes_bytes, uint64_t scale_bytes, unsigned* err) {
@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(256) mx_quantize_kernel(const void* __restrict
       live[u] = t < total_items;
       const int64_t pb = t >> 1;
       h[u] = (int)(t & 1);
-      r[u] = pb / nblk_pad;
+      r[u] = div_u32((uint32_t)pb, div_nblk_pad);   // pb < 2^31 (checked on the host)
       j[u] = pb - r[u] * nblk_pad;
       real[u] = live[u] && r[u] < M && j[u] < nblk;
       if (real[u]) load_block<kF32>(x, (uint32_t)(r[u] * (K / 16) + 2 * j[u] + h[u]), B[u]);
@@ -117,7 +117,8 @@ nvfp4_status nvfp4_mx_quantize(const void* x, nvfp4_in_dtype dtype, int64_t M, i
   const int64_t rows = tc ? ceil_div(M, 128) * 128 : M;
   const int64_t nblk_pad = tc ? 4 * kc : K / 32;
   const int64_t total = rows * nblk_pad * 2;
-  // one pass over the tensor, two items per thread (as the NVFP4 quantizer)
+  // one pass over the tensor, two items per thread (L2-cold 4096x5120 bf16:
+  // 13.4 us against 15.3 us for a persistent grid of 4 CTAs per SM)
   const int blocks = (int)std::max<int64_t>(1, ceil_div(total, 512));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(blocks);
@@ -129,13 +130,14 @@ nvfp4_status nvfp4_mx_quantize(const void* x, nvfp4_in_dtype dtype, int64_t M, i
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const bool f32 = dtype == NVFP4_IN_F32;
+  const DivU32 div_np = make_div((uint32_t)nblk_pad);
   const uint64_t codes_bytes = (uint64_t)M * (uint64_t)(K / 2);
   const uint64_t scale_bytes = tc ? (uint64_t)(rows / 128) * kc * 512 : (uint64_t)M * (uint64_t)(K / 32);
   cudaError_t e;
-  if (f32) e = tc ? cudaLaunchKernelEx(&cfg, mx_quantize_kernel<true, true>, x, M, K, nblk_pad, total, codes, scales, kc, codes_bytes, scale_bytes, d->err_word)
-                  : cudaLaunchKernelEx(&cfg, mx_quantize_kernel<true, false>, x, M, K, nblk_pad, total, codes, scales, kc, codes_bytes, scale_bytes, d->err_word);
-  else e = tc ? cudaLaunchKernelEx(&cfg, mx_quantize_kernel<false, true>, x, M, K, nblk_pad, total, codes, scales, kc, codes_bytes, scale_bytes, d->err_word)
-              : cudaLaunchKernelEx(&cfg, mx_quantize_kernel<false, false>, x, M, K, nblk_pad, total, codes, scales, kc, codes_bytes, scale_bytes, d->err_word);
+  if (f32) e = tc ? cudaLaunchKernelEx(&cfg, mx_quantize_kernel<true, true>, x, M, K, nblk_pad, div_np, total, codes, scales, kc, codes_bytes, scale_bytes, d->err_word)
+                  : cudaLaunchKernelEx(&cfg, mx_quantize_kernel<true, false>, x, M, K, nblk_pad, div_np, total, codes, scales, kc, codes_bytes, scale_bytes, d->err_word);
+  else e = tc ? cudaLaunchKernelEx(&cfg, mx_quantize_kernel<false, true>, x, M, K, nblk_pad, div_np, total, codes, scales, kc, codes_bytes, scale_bytes, d->err_word)
+              : cudaLaunchKernelEx(&cfg, mx_quantize_kernel<false, false>, x, M, K, nblk_pad, div_np, total, codes, scales, kc, codes_bytes, scale_bytes, d->err_word);
   return cuda_status(e);
 }
 

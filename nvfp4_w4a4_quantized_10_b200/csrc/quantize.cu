@@ -25,19 +25,6 @@ __device__ __forceinline__ int64_t tc_scale_offset(int64_t r, int64_t j, int64_t
   return ((r >> 7) * kc + (j >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (j & 3);
 }
 
-// Unsigned division by an invariant divisor d (Granlund and Montgomery,
-// "Division by invariant integers using multiplication", 1994, unsigned
-// case): with l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1,
-// n / d == (mulhi(n, m) + n) >> l for every 32-bit n.
-struct DivU32 {
-  uint32_t m, l;
-};
-
-__device__ __forceinline__ uint32_t div_u32(uint32_t n, DivU32 d) {
-  const uint32_t t = __umulhi(n, d.m);
-  return (uint32_t)(((uint64_t)t + n) >> d.l);
-}
-
 // Raise *amax to v.  Non-negative floats order like their bit patterns, so
 // an unsigned atomic maximum does it; the word only grows while the kernel
 // runs, so a CTA whose maximum is not above a value it reads there has
@@ -228,14 +215,6 @@ int grid_for(int64_t work_items, int threads, const DeviceInfo* d, int per_sm = 
   return (int)blocks;
 }
 
-DivU32 make_div(uint32_t d) {
-  uint32_t l = 0;
-  while ((1ull << l) < d) ++l;
-  DivU32 r;
-  r.l = l;
-  r.m = (uint32_t)((((1ull << l) - d) << 32) / d + 1);
-  return r;
-}
 
 template <bool kF32, bool kTC, bool kAmax>
 cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, float g, uint8_t* codes, uint8_t* scales,
