@@ -176,8 +176,9 @@ NVFP4_API nvfp4_status nvfp4_swizzle_scales(const uint8_t* rowmajor, int64_t row
  * calls on different streams use different workspaces.  Each launch leaves
  * the words it used empty (zero), so a workspace stays ready for the next.
  * M > 128 uses no workspace.
- * Co-residency: the split-K grid has one CTA per SM of the device
- * (multiProcessorCount), and the CTA that sums a split tile waits (bounded)
+ * Co-residency: the split-K grid has two CTAs per SM of the device
+ * (multiProcessorCount) for M <= 16 and one per SM for 16 < M <= 128, and
+ * the CTA that sums a split tile waits (bounded)
  * for partials from CTAs with higher indices.  So every CTA of the grid must
  * be able to run at the same time.  That holds when the call has the whole
  * GPU.  It does not hold when the process is limited to fewer SMs than the
@@ -197,9 +198,10 @@ NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scale
                         nvfp4_stream_t stream);
 
 /* Bytes of K-split workspace nvfp4_gemm / nvfp4_linear need on the current
- * device for an M x N x K problem: 2 * SMs * BN * 128 * 8, BN being the
+ * device for an M x N x K problem: 2 * CTAs * BN * 128 * 8, BN being the
  * activation tile width the call picks (16, 32, 64 or 128 for M <= 16, 32,
- * 64, 128); 0 for M > 128 (no split) or invalid sizes.  No counterpart in
+ * 64, 128) and CTAs the split-K grid (2 * SMs for BN = 16, SMs otherwise);
+ * 0 for M > 128 (no split) or invalid sizes.  No counterpart in
  * the pages: the sizing rule of this library's split-K exchange.
  * nvfp4_workspace_bytes(128, N, K) (2 * SMs * 128 KB) covers every shape. */
 NVFP4_API size_t nvfp4_workspace_bytes(int64_t M, int64_t N, int64_t K);

@@ -133,7 +133,7 @@ struct Cfg {
   static constexpr int kOutBytes = SWAP ? 0 : 2 * kStageOutBytes;    // double-buffered output sub-tiles
   // in-kernel activation: codes (BN rows x 128 B, 128B swizzle) and one
   // 128-row scale block per K-step, for up to kActSteps steps
-  static constexpr int kActSteps = kQx ? 16 : 0;
+  static constexpr int kActSteps = kQx ? (BN <= 16 ? 8 : 16) : 0;
   static constexpr int kActCodeBytes = BN * kRowBytes;
   static constexpr int kActSfBytes = kKB * kSfChunk;
   static constexpr int kActBytes = kActSteps * (kActCodeBytes + kActSfBytes);
@@ -141,13 +141,18 @@ struct Cfg {
   // prefill and fused shape measured (the deeper ring lets the copy warps
   // run further ahead of MMAs that are not waiting on data)
   static constexpr int kMaxStages = PAIR ? 4 : 8;
-  // Decode tiles with a small activation side run two CTAs per SM: the next
-  // GEMM on the stream (programmatic dependent launch) then starts at once
-  // beside this one and streams its weight while this one finishes, instead
-  // of waiting for this grid's CTAs to leave.  Each CTA keeps to half of the
-  // SM's shared memory (and TMEM and registers).
-  static constexpr bool kCoRes = SWAP && !kQx && BN <= 32;
+  // Decode tiles with a small activation side fit two CTAs per SM, each
+  // keeping to half of the SM's shared memory (and TMEM and registers).  With
+  // BN = 16 the grid itself has two CTAs per SM: each streams half as much
+  // weight, and each SM has twice the stages in flight (decode step 12.4
+  // against 13.3 us at 8x12288x5120).  With BN = 32 (slower at two per SM)
+  // the grid has one per SM, and the second slot lets the next GEMM on the
+  // stream start beside it (programmatic dependent launch).  The in-kernel
+  // activation variant follows the same grid (its BN = 16 form holds 8
+  // K-steps of activation instead of 16, covering the same shapes).
+  static constexpr bool kCoRes = SWAP && (kQx ? BN <= 16 : BN <= 32);
   static constexpr int kMinBlocks = kCoRes ? 2 : 1;
+  static constexpr int kGridPerSm = SWAP && BN <= 16 ? 2 : 1;
   static constexpr int kSmemBudget = kCoRes ? 112 * 1024 : 222 * 1024;
   static constexpr int kFit = (kSmemBudget - kOutBytes - kActBytes) / kStageBytes;
   static constexpr int kStages = kFit < kMaxStages ? kFit : kMaxStages;
@@ -1215,9 +1220,13 @@ struct Workspace {
 std::mutex g_ws_mu;
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws_table;
 
-// Bytes of K-split workspace a swapped GEMM with activation side bn needs.
+// CTAs of a swapped GEMM's grid, at most (Cfg::kGridPerSm per SM).
+int64_t swap_grid_cap(const DeviceInfo* d, int bn) { return (int64_t)d->sm_count * (bn <= 16 ? 2 : 1); }
+
+// Bytes of K-split workspace a swapped GEMM with activation side bn needs:
+// two slots of bn x 128 words per CTA.
 size_t workspace_need(const DeviceInfo* d, int bn) {
-  return (size_t)2 * d->sm_count * (size_t)bn * kBM * sizeof(uint64_t);
+  return (size_t)2 * (size_t)swap_grid_cap(d, bn) * (size_t)bn * kBM * sizeof(uint64_t);
 }
 
 cudaError_t get_workspace(const DeviceInfo* d, cudaStream_t st, int bn, Workspace* out) {
@@ -1267,7 +1276,8 @@ cudaError_t launch(const GemmParams& p, const DeviceInfo* d, cudaStream_t st, in
   if (grid == 0) {
     if (SWAP) {
       const int64_t units = (int64_t)p.tiles_p * p.kt;
-      grid = (int)(units < d->sm_count ? units : d->sm_count);
+      const int64_t cap = (int64_t)d->sm_count * Cf::kGridPerSm;
+      grid = (int)(units < cap ? units : cap);
     } else {
       const int tiles = p.tiles_p * p.tiles_q;
       grid = tiles < d->sm_count ? tiles : d->sm_count;
@@ -1463,16 +1473,20 @@ uint8_t* noalloc_scratch_ptr(int device) {
 // writes (a_codes, a_scales) and the GEMM reads them.  Without them,
 // decode-sized M runs as one kernel whose epilogue warps quantize X into
 // shared memory before the first MMA.  (That one-kernel form measured slower
-// than the two kernels on the decode shape, 15.7 vs 12.9 us: the 148 CTAs
-// each quantize most of X again, in four warps that cannot hide latency,
-// whereas the quantize kernel spreads X over the whole GPU once.)
+// than the two kernels on the decode shape: every CTA quantizes the part of
+// X its K range needs, so X is quantized many times over, in four warps that
+// cannot hide latency, whereas the quantize kernel spreads X over the whole
+// GPU once.)
 constexpr int kLinearMaxM = 32;
 
 bool linear_fused_fits(const DeviceInfo* d, int64_t M, int64_t N, int64_t K) {
   if (M > kLinearMaxM) return false;
+  const int bn = M <= 16 ? 16 : 32;
   const int64_t units = ceil_div(N, kBM) * ceil_div(K, 64 * Cfg<16, true>::kKB);
-  const int64_t grid = units < d->sm_count ? units : d->sm_count;
-  return ceil_div(units, grid) <= Cfg<16, true, 1>::kActSteps;   // steps per CTA, at most
+  const int64_t cap = swap_grid_cap(d, bn);
+  const int64_t grid = units < cap ? units : cap;
+  const int steps = bn == 16 ? Cfg<16, true, 1>::kActSteps : Cfg<32, true, 1>::kActSteps;
+  return ceil_div(units, grid) <= steps;   // steps per CTA, at most
 }
 
 template <int BN, int QX>
@@ -1597,6 +1611,9 @@ nvfp4_status run_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_scales, f
   GemmParams p;
   std::memset(&p, 0, sizeof(p));
   const int bn = M <= 16 ? 16 : 32;
+  // the grid's partial slots fit the scratch: 2 x (2 x SMs) x 16 x 128 words
+  // for bn = 16, 2 x SMs x 32 x 128 for bn = 32; both fit for <= 160 SMs
+  if (workspace_need(d, bn) > kNoAllocScratchBytes) return NVFP4_ERR_UNSUPPORTED;
   p.ws = reinterpret_cast<uint64_t*>(scratch);
   p.ws_words = kNoAllocScratchBytes / sizeof(uint64_t);
   p.rows_p = (int)N;

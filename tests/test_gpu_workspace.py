@@ -33,8 +33,10 @@ def _problem(M, N, K, seed):
 
 def test_workspace_bytes_rule():
     sm = torch.cuda.get_device_properties(0).multi_processor_count
+    # two slots of bn x 128 words per CTA; the bn = 16 grid has two CTAs per SM
     for M, bn in ((1, 16), (16, 16), (17, 32), (32, 32), (33, 64), (64, 64), (65, 128), (128, 128)):
-        assert nv.nvfp4_workspace_bytes(M, 4096, 1024) == 2 * sm * bn * 128 * 8, M
+        ctas = 2 * sm if bn == 16 else sm
+        assert nv.nvfp4_workspace_bytes(M, 4096, 1024) == 2 * ctas * bn * 128 * 8, M
     assert nv.nvfp4_workspace_bytes(129, 4096, 1024) == 0
     assert nv.nvfp4_workspace_bytes(0, 4096, 1024) == 0
     assert nv.nvfp4_workspace_bytes(8, 4096, 48) == 0

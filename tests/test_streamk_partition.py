@@ -27,7 +27,8 @@ def items(c, U, G, kt):
 
 
 @pytest.mark.parametrize("tiles,kt,G", [(96, 20, 148), (96, 20, 96), (1, 20, 20), (1, 3, 3), (7, 5, 148),
-                                        (200, 20, 148), (3, 1, 3), (13, 7, 148), (1000, 20, 148), (96, 68, 148)])
+                                        (200, 20, 148), (3, 1, 3), (13, 7, 148), (1000, 20, 148), (96, 68, 148),
+                                        (96, 20, 296), (96, 68, 296), (40, 3, 296)])
 def test_partition(tiles, kt, G):
     U = tiles * kt
     G = min(G, U)
@@ -62,7 +63,7 @@ def test_partition(tiles, kt, G):
 
 def test_cta_of_unit_inverts_unit_begin():
     for U in (1, 7, 1920, 9999):
-        for G in (1, 3, 148):
+        for G in (1, 3, 148, 296):
             if G > U:
                 continue
             for u in range(U):
