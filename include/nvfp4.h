@@ -176,18 +176,21 @@ NVFP4_API nvfp4_status nvfp4_swizzle_scales(const uint8_t* rowmajor, int64_t row
  * calls on different streams use different workspaces.  Each launch leaves
  * the words it used empty (zero), so a workspace stays ready for the next.
  * M > 128 uses no workspace.
- * Co-residency: the split-K grid has two CTAs per SM of the device
- * (multiProcessorCount) for M <= 16 and one per SM for 16 < M <= 128, and
- * the CTA that sums a split tile waits (bounded)
- * for partials from CTAs with higher indices.  So every CTA of the grid must
- * be able to run at the same time.  That holds when the call has the whole
- * GPU.  It does not hold when the process is limited to fewer SMs than the
- * device reports (an MPS active-thread percentage, a green context, or
- * another kernel occupying SMs for longer than the wait bound).  Then the
- * waits run out and the call reports NVFP4_ERR_TIMEOUT through
- * nvfp4_last_device_error (nothing hangs).  nvfp4_set_decode_cooperative(1)
- * makes the driver guarantee co-residency: it launches the grid
- * cooperatively or refuses it (UNSUPPORTED), at about 1.5 us per call.
+ * Progress of the split-K grid: the grid has 2 x SMs CTAs
+ * (multiProcessorCount) for M <= 16, which the GPU runs as two waves (one
+ * CTA of this kernel is resident per SM), and SMs CTAs for 16 < M <= 128.
+ * The CTA that sums a split tile waits (bounded) only for partials that
+ * CTAs with higher indices produce as their first work item.  So the grid
+ * completes when its CTAs start in index order, as the hardware does when
+ * the call has the GPU to itself.  If the process is limited to fewer SMs
+ * than the device reports (an MPS active-thread percentage, a green context)
+ * or CTAs start out of order, a wait can run out: the call then reports
+ * NVFP4_ERR_TIMEOUT through nvfp4_last_device_error, and nothing hangs.
+ * nvfp4_set_decode_cooperative(1) removes the assumption.  The grid is then
+ * sized to the CTAs that can be resident at once (occupancy API) and
+ * launched cooperatively, which the driver admits only if they all fit
+ * (else UNSUPPORTED).  For M <= 16 that grid is smaller than the default, so
+ * the K split and the FP32 summation order differ from the default launch.
  * Errors: INVALID_ARG (also: a registered workspace smaller than
  * nvfp4_workspace_bytes for this shape), ALIGNMENT, UNSUPPORTED (device is
  * not sm_100, or a first decode-shaped call during capture with no
@@ -416,11 +419,15 @@ NVFP4_API void nvfp4_set_wait_timeout_ns(uint64_t ns);
 /* Launch the split-K (decode, M <= 128) grids of nvfp4_gemm, nvfp4_linear,
  * nvfp4_gemm_noalloc, nvfp4_fused_proj and nvfp4_mx_gemm as cooperative
  * grids (enable != 0) from now on, process-wide; 0 (the default) restores
- * ordinary launches.  A cooperative grid is admitted only if all of its CTAs
- * can be resident at once, which the split-K reduction needs (see
- * nvfp4_gemm); a grid that cannot be returns UNSUPPORTED instead of timing
- * out.  Results are bitwise the same either way.  Costs about 1.5 us per
- * decode GEMM on B200.  No counterpart in the pages. */
+ * ordinary launches.  A cooperative grid is sized to the CTAs the occupancy
+ * API admits per SM and is admitted by the driver only if all of them can be
+ * resident at once, which guarantees the split-K reduction's progress
+ * without relying on the order in which CTAs start (see nvfp4_gemm).  A grid
+ * that cannot be resident returns UNSUPPORTED instead of timing out.  For
+ * M > 16 results are bitwise those of the default launch; for M <= 16 the
+ * grid is smaller, so they match up to FP32 summation order.  nvfp4_linear
+ * without activation buffers then covers fewer shapes: one CTA per SM must
+ * hold its K range in 8 steps for M <= 16.  No counterpart in the pages. */
 NVFP4_API void nvfp4_set_decode_cooperative(int enable);
 
 /* 1 if this is the bounds-checked debug build (libnvfp4_debug.so, compiled

@@ -141,19 +141,25 @@ struct Cfg {
   // prefill and fused shape measured (the deeper ring lets the copy warps
   // run further ahead of MMAs that are not waiting on data)
   static constexpr int kMaxStages = PAIR ? 4 : 8;
-  // Decode tiles with a small activation side fit two CTAs per SM, each
-  // keeping to half of the SM's shared memory (and TMEM and registers).  With
-  // BN = 16 the grid itself has two CTAs per SM: each streams half as much
-  // weight, and each SM has twice the stages in flight (decode step 12.4
-  // against 13.3 us at 8x12288x5120).  With BN = 32 (slower at two per SM)
-  // the grid has one per SM, and the second slot lets the next GEMM on the
-  // stream start beside it (programmatic dependent launch).  The in-kernel
-  // activation variant follows the same grid (its BN = 16 form holds 8
-  // K-steps of activation instead of 16, covering the same shapes).
+  // Decode tiles with a small activation side keep to under half of the
+  // SM's shared memory (and TMEM, and 128 registers).  The occupancy API
+  // still reports one resident CTA per SM for this kernel (at 91 KB as at
+  // 114 KB), so with BN = 16 the grid of 2 x SMs CTAs runs as two waves: a
+  // second-wave CTA starts streaming on an SM as soon as the first-wave CTA
+  // there is done, which overlaps that CTA's split-K tail (decode step 12.4
+  // against 13.3 us at 8x12288x5120; four stages measured 2 % faster than
+  // five).  A split tile's summing CTA waits only for partials that CTAs
+  // with higher indices produce as their first work item, so the waves make
+  // progress when CTAs start in index order (bounded waits report a timeout
+  // otherwise); the opt-in cooperative launch sizes the grid to what is
+  // resident instead.  BN = 32 is slower in two waves and keeps one CTA per
+  // SM.  The in-kernel activation variant follows the same grid (its
+  // BN = 16 form holds 8 K-steps of activation instead of 16, covering the
+  // same shapes).
   static constexpr bool kCoRes = SWAP && (kQx ? BN <= 16 : BN <= 32);
   static constexpr int kMinBlocks = kCoRes ? 2 : 1;
   static constexpr int kGridPerSm = SWAP && BN <= 16 ? 2 : 1;
-  static constexpr int kSmemBudget = kCoRes ? 112 * 1024 : 222 * 1024;
+  static constexpr int kSmemBudget = kCoRes ? 104 * 1024 : 222 * 1024;
   static constexpr int kFit = (kSmemBudget - kOutBytes - kActBytes) / kStageBytes;
   static constexpr int kStages = kFit < kMaxStages ? kFit : kMaxStages;
   static constexpr int kOffA = 0;
@@ -201,7 +207,7 @@ struct Cfg {
   static_assert(kAcc1Col % 32 == 0, "accumulator column alignment");
   static_assert(kStages >= 2, "pipeline depth");
   static_assert(kSfBase + kSfRegions * kSfStageCols <= kTmemAlloc, "TMEM budget");
-  static_assert(!kCoRes || kSmemBytes <= 113 * 1024, "two CTAs per SM");
+  static_assert(!kCoRes || kSmemBytes <= 113 * 1024, "under half of the SM's shared memory");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(BN % 16 == 0 && BN <= 256, "MMA N");
   static_assert(!kQx || (SWAP && BN <= 32), "in-kernel activation: swapped tiles, M <= 32");
@@ -1260,10 +1266,34 @@ cudaError_t set_smem_attr(const DeviceInfo* d) {
   static std::once_flag once[64];
   static cudaError_t attr_err[64];
   std::call_once(once[d->device], [&] {
-    attr_err[d->device] = cudaFuncSetAttribute(nvfp4_gemm_kernel<BN, SWAP, OUT_F32, QX, MX, PAIR>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmemBytes);
+    auto kern = nvfp4_gemm_kernel<BN, SWAP, OUT_F32, QX, MX, PAIR>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmemBytes);
+    // all of the SM's unified memory as shared memory: two co-resident CTAs
+    // of 114 KB fit only with the full carveout, and a cooperative launch is
+    // admitted against this preference
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    attr_err[d->device] = e;
   });
   return attr_err[d->device];
+}
+
+// CTAs of this kernel that can be resident on one SM (occupancy API, with the
+// attributes set above), once per device; 0 if the query fails.
+template <int BN, bool SWAP, bool OUT_F32, int QX = 0, bool MX = false, bool PAIR = false>
+int resident_per_sm(const DeviceInfo* d) {
+  using Cf = Cfg<BN, SWAP, QX, MX, PAIR>;
+  static std::once_flag once[64];
+  static int occ[64];
+  std::call_once(once[d->device], [&] {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, nvfp4_gemm_kernel<BN, SWAP, OUT_F32, QX, MX, PAIR>,
+                                                      Cf::kThreads, Cf::kSmemBytes) != cudaSuccess) {
+      (void)cudaGetLastError();
+      n = 0;
+    }
+    occ[d->device] = n;
+  });
+  return occ[d->device];
 }
 
 // grid: number of CTAs (0 = the persistent grid); cluster: CTAs per cluster
@@ -1276,7 +1306,14 @@ cudaError_t launch(const GemmParams& p, const DeviceInfo* d, cudaStream_t st, in
   if (grid == 0) {
     if (SWAP) {
       const int64_t units = (int64_t)p.tiles_p * p.kt;
-      const int64_t cap = (int64_t)d->sm_count * Cf::kGridPerSm;
+      int per_sm = Cf::kGridPerSm;
+      if (decode_cooperative()) {
+        // a cooperative grid must be resident at once: at most what the
+        // occupancy API admits per SM
+        const int occ = resident_per_sm<BN, SWAP, OUT_F32, QX, MX, PAIR>(d);
+        if (occ < per_sm) per_sm = occ < 1 ? 1 : occ;
+      }
+      const int64_t cap = (int64_t)d->sm_count * per_sm;
       grid = (int)(units < cap ? units : cap);
     } else {
       const int tiles = p.tiles_p * p.tiles_q;
@@ -1483,7 +1520,8 @@ bool linear_fused_fits(const DeviceInfo* d, int64_t M, int64_t N, int64_t K) {
   if (M > kLinearMaxM) return false;
   const int bn = M <= 16 ? 16 : 32;
   const int64_t units = ceil_div(N, kBM) * ceil_div(K, 64 * Cfg<16, true>::kKB);
-  const int64_t cap = swap_grid_cap(d, bn);
+  // a cooperative grid may be as small as one CTA per SM (see launch())
+  const int64_t cap = decode_cooperative() ? (int64_t)d->sm_count : swap_grid_cap(d, bn);
   const int64_t grid = units < cap ? units : cap;
   const int steps = bn == 16 ? Cfg<16, true, 1>::kActSteps : Cfg<32, true, 1>::kActSteps;
   return ceil_div(units, grid) <= steps;   // steps per CTA, at most

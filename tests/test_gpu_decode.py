@@ -123,36 +123,40 @@ def test_decode_mxfp4(M, N, K):
     assert torch.equal(out16, out32.to(torch.bfloat16))
 
 
-@pytest.mark.parametrize("M,N,K", [(8, 12288, 5120), (16, 4097, 1024), (64, 1000, 2048), (128, 3000, 768)])
-def test_decode_cooperative_launch_is_bitwise_equal(M, N, K):
-    # the opt-in co-residency guarantee changes how the grid is launched, not
-    # what it computes: same K split, same summation order
+@pytest.mark.parametrize("M,N,K", [(8, 12288, 5120), (16, 4097, 1024), (24, 3000, 5120), (64, 1000, 2048),
+                                   (128, 3000, 768)])
+def test_decode_cooperative_launch(M, N, K):
+    # The opt-in co-residency guarantee launches the split-K grid
+    # cooperatively, sized to what the occupancy API admits per SM.  Where
+    # that is the default grid (M > 16) the result is bitwise the default's;
+    # for M <= 16 the default grid has two CTAs per SM, more than are
+    # resident at once, so the cooperative grid can split K differently:
+    # the same sum up to FP32 rounding order.
     (ac, asc, ga), (wc, wsc, gw) = _operands(M, N, K, seed=7 * M + K)
     a_d, as_d = to_dev_operand(ac, asc, K)
     w_d, ws_d = to_dev_operand(wc, wsc, K)
     default = gpu_gemm(a_d, as_d, ga, w_d, ws_d, gw, M, N, K, torch.float32)
-    x = torch.from_numpy(synth.student_t_outliers(M, K, seed=M, dtype=torch.float32).numpy()).to(DEV)
-    lin_default = torch.empty(M, N, dtype=torch.bfloat16, device=DEV)
-    if M <= 32:
-        nv.nvfp4_linear(x, float(ga), w_d, ws_d, float(gw), N, lin_default)
     torch.cuda.synchronize()
     nv.nvfp4_set_decode_cooperative(True)
     try:
         coop = gpu_gemm(a_d, as_d, ga, w_d, ws_d, gw, M, N, K, torch.float32)
+        again = gpu_gemm(a_d, as_d, ga, w_d, ws_d, gw, M, N, K, torch.float32)
         if M <= 32:
-            lin = torch.empty_like(lin_default)
-            nv.nvfp4_linear(x, float(ga), w_d, ws_d, float(gw), N, lin)
             noalloc = torch.empty(M, N, dtype=torch.float32, device=DEV)
             nv.nvfp4_gemm_noalloc(a_d, as_d, float(ga), w_d, ws_d, float(gw), M, N, K, noalloc)
         torch.cuda.synchronize()
     finally:
         nv.nvfp4_set_decode_cooperative(False)
     check_device_error_word()
-    assert torch.equal(coop, default)
-    assert_gemm_close(coop.cpu().numpy(), oracle.gemm(ac, asc, ga, wc, wsc, gw), f"cooperative {M}x{N}x{K}")
+    assert torch.equal(coop, again)
     if M <= 32:
-        assert torch.equal(lin, lin_default)
-        assert torch.equal(noalloc, default)
+        assert torch.equal(noalloc, coop)          # the same cooperative grid
+    assert_gemm_close(coop.cpu().numpy(), oracle.gemm(ac, asc, ga, wc, wsc, gw), f"cooperative {M}x{N}x{K}")
+    if M > 16:
+        assert torch.equal(coop, default)
+    else:
+        max_rel, frob = rel_errors(coop.double().cpu().numpy(), default.double().cpu().numpy())
+        assert max_rel <= TOL_MAX_REL and frob <= TOL_FROB, (max_rel, frob)
 
 
 @pytest.mark.parametrize("M,N,K", [(8, 12288, 5120), (16, 2048, 4096), (4, 700, 17408)])
