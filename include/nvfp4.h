@@ -177,8 +177,8 @@ NVFP4_API nvfp4_status nvfp4_swizzle_scales(const uint8_t* rowmajor, int64_t row
  * the words it used empty (zero), so a workspace stays ready for the next.
  * M > 128 uses no workspace.
  * Progress of the split-K grid: the grid has 2 x SMs CTAs
- * (multiProcessorCount) for M <= 16, which the GPU runs as two waves (one
- * CTA of this kernel is resident per SM), and SMs CTAs for 16 < M <= 128.
+ * (multiProcessorCount) for M <= 16, two per SM, and SMs CTAs for
+ * 16 < M <= 128.
  * The CTA that sums a split tile waits (bounded) only for partials that
  * CTAs with higher indices produce as their first work item.  So the grid
  * completes when its CTAs start in index order, as the hardware does when

@@ -142,18 +142,18 @@ struct Cfg {
   // run further ahead of MMAs that are not waiting on data)
   static constexpr int kMaxStages = PAIR ? 4 : 8;
   // Decode tiles with a small activation side keep to under half of the
-  // SM's shared memory (and TMEM, and 128 registers).  The occupancy API
-  // still reports one resident CTA per SM for this kernel (at 91 KB as at
-  // 114 KB), so with BN = 16 the grid of 2 x SMs CTAs runs as two waves: a
-  // second-wave CTA starts streaming on an SM as soon as the first-wave CTA
-  // there is done, which overlaps that CTA's split-K tail (decode step 12.4
+  // SM's shared memory (and TMEM, and 128 registers), so two CTAs fit on an
+  // SM.  With BN = 16 the grid has 2 x SMs CTAs: each streams half as much
+  // weight and each SM keeps twice the stages in flight (decode step 12.4
   // against 13.3 us at 8x12288x5120; four stages measured 2 % faster than
-  // five).  A split tile's summing CTA waits only for partials that CTAs
-  // with higher indices produce as their first work item, so the waves make
-  // progress when CTAs start in index order (bounded waits report a timeout
-  // otherwise); the opt-in cooperative launch sizes the grid to what is
-  // resident instead.  BN = 32 is slower in two waves and keeps one CTA per
-  // SM.  The in-kernel activation variant follows the same grid (its
+  // five).  The profiler's occupancy limits are two CTAs per SM and it sees
+  // about 1.8 resident on average, but the occupancy API reports one.  A
+  // split tile's summing CTA waits only for partials that CTAs with higher
+  // indices produce as their first work item, so the grid completes whenever
+  // CTAs start in index order, resident together or not (bounded waits
+  // report a timeout otherwise); the opt-in cooperative launch sizes the
+  // grid to what the occupancy API admits instead.  BN = 32 is slower at two
+  // per SM and keeps one CTA per SM.  The in-kernel activation variant follows the same grid (its
   // BN = 16 form holds 8 K-steps of activation instead of 16, covering the
   // same shapes).
   static constexpr bool kCoRes = SWAP && (kQx ? BN <= 16 : BN <= 32);
