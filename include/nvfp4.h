@@ -178,7 +178,7 @@ NVFP4_API nvfp4_status nvfp4_swizzle_scales(const uint8_t* rowmajor, int64_t row
  * M > 128 uses no workspace.
  * Progress of the split-K grid: the grid has 2 x SMs CTAs
  * (multiProcessorCount) for M <= 16, two per SM, and SMs CTAs for
- * 16 < M <= 128.
+ * 16 < M <= 128 (and for every MXFP4 GEMM).
  * The CTA that sums a split tile waits (bounded) only for partials that
  * CTAs with higher indices produce as their first work item.  So the grid
  * completes when its CTAs start in index order, as the hardware does when
@@ -203,7 +203,8 @@ NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scale
 /* Bytes of K-split workspace nvfp4_gemm / nvfp4_linear need on the current
  * device for an M x N x K problem: 2 * CTAs * BN * 128 * 8, BN being the
  * activation tile width the call picks (16, 32, 64 or 128 for M <= 16, 32,
- * 64, 128) and CTAs the split-K grid (2 * SMs for BN = 16, SMs otherwise);
+ * 64, 128) and CTAs the NVFP4 split-K grid (2 * SMs for BN = 16, SMs
+ * otherwise; the MXFP4 grid is SMs, so this size covers it too);
  * 0 for M > 128 (no split) or invalid sizes.  No counterpart in
  * the pages: the sizing rule of this library's split-K exchange.
  * nvfp4_workspace_bytes(128, N, K) (2 * SMs * 128 KB) covers every shape. */

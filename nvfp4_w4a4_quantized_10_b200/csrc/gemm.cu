@@ -152,13 +152,14 @@ struct Cfg {
   // indices produce as their first work item, so the grid completes whenever
   // CTAs start in index order, resident together or not (bounded waits
   // report a timeout otherwise); the opt-in cooperative launch sizes the
-  // grid to what the occupancy API admits instead.  BN = 32 is slower at two
-  // per SM and keeps one CTA per SM.  The in-kernel activation variant follows the same grid (its
+  // grid to what the occupancy API admits instead.  BN = 32, and the MXFP4
+  // decode tile (13.5 against 10.9 us), are slower at two per SM and keep
+  // one CTA per SM.  The in-kernel activation variant follows the same grid (its
   // BN = 16 form holds 8 K-steps of activation instead of 16, covering the
   // same shapes).
   static constexpr bool kCoRes = SWAP && (kQx ? BN <= 16 : BN <= 32);
   static constexpr int kMinBlocks = kCoRes ? 2 : 1;
-  static constexpr int kGridPerSm = SWAP && BN <= 16 ? 2 : 1;
+  static constexpr int kGridPerSm = SWAP && BN <= 16 && !MX ? 2 : 1;
   static constexpr int kSmemBudget = kCoRes ? 104 * 1024 : 222 * 1024;
   static constexpr int kFit = (kSmemBudget - kOutBytes - kActBytes) / kStageBytes;
   static constexpr int kStages = kFit < kMaxStages ? kFit : kMaxStages;
@@ -1226,7 +1227,8 @@ struct Workspace {
 std::mutex g_ws_mu;
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws_table;
 
-// CTAs of a swapped GEMM's grid, at most (Cfg::kGridPerSm per SM).
+// CTAs of a swapped GEMM's grid, at most (Cfg::kGridPerSm per SM; the
+// NVFP4 bound, which also covers the MXFP4 grid).
 int64_t swap_grid_cap(const DeviceInfo* d, int bn) { return (int64_t)d->sm_count * (bn <= 16 ? 2 : 1); }
 
 // Bytes of K-split workspace a swapped GEMM with activation side bn needs:
