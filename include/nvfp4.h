@@ -428,7 +428,9 @@ NVFP4_API void nvfp4_set_wait_timeout_ns(uint64_t ns);
  * M > 16 results are bitwise those of the default launch; for M <= 16 the
  * grid is smaller, so they match up to FP32 summation order.  nvfp4_linear
  * without activation buffers then covers fewer shapes: one CTA per SM must
- * hold its K range in 8 steps for M <= 16.  No counterpart in the pages. */
+ * hold its K range in 8 steps for M <= 16.  The setting is read when a call
+ * is made: change it only while no library call is being made on another
+ * host thread.  No counterpart in the pages. */
 NVFP4_API void nvfp4_set_decode_cooperative(int enable);
 
 /* 1 if this is the bounds-checked debug build (libnvfp4_debug.so, compiled
