@@ -160,8 +160,7 @@ struct Cfg {
   static constexpr bool kCoRes = SWAP && (kQx ? BN <= 16 : BN <= 32);
   static constexpr int kMinBlocks = kCoRes ? 2 : 1;
   static constexpr int kGridPerSm = SWAP && BN <= 16 && !MX ? 2 : 1;
-  // the two-per-SM NVFP4 decode tile keeps 3 stages (2 % faster than 4)
-  static constexpr int kSmemBudget = (kGridPerSm == 2 && !kQx) ? 80 * 1024 : kCoRes ? 104 * 1024 : 222 * 1024;
+  static constexpr int kSmemBudget = kCoRes ? 104 * 1024 : 222 * 1024;
   static constexpr int kFit = (kSmemBudget - kOutBytes - kActBytes) / kStageBytes;
   static constexpr int kStages = kFit < kMaxStages ? kFit : kMaxStages;
   static constexpr int kOffA = 0;
@@ -185,12 +184,7 @@ struct Cfg {
   static constexpr int kOffSeg = kOffBar + kNumBars * 8;             // segment table: ends, alphas
   static constexpr int kOffMisc = kOffSeg + 2 * 4 * NVFP4_MAX_SEGMENTS;
   static constexpr int kOffRtab = kOffMisc + 16;                     // in-kernel activation: g / e4m3(s)
-  static constexpr int kSmemUsed = kOffRtab + (kQx ? 1024 : 0) + 1024;   // + alignment slack
-  // the two-per-SM decode tile asks for at least 78 KB, so that shared
-  // memory alone keeps a third CTA off the SM (three would need more TMEM
-  // than the SM has: each allocates 256 columns)
-  static constexpr int kSmemFloor = (kGridPerSm == 2 && !kQx) ? 78 * 1024 : 0;
-  static constexpr int kSmemBytes = kSmemUsed > kSmemFloor ? kSmemUsed : kSmemFloor;
+  static constexpr int kSmemBytes = kOffRtab + (kQx ? 1024 : 0) + 1024;   // + alignment slack
   // TMEM columns.  Normal 128x256 tiles: the copy warps run ahead of the
   // MMAs, so the scales of successive steps use a ring of regions at the top
   // of TMEM ([320,512) for four 48-column regions); the two accumulator
