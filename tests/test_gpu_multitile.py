@@ -1,12 +1,13 @@
 """Persistent multi-tile GEMM paths at the stated FP32 tolerance, on all rows.
 
-The prefill-shaped kernel runs one persistent CTA per SM over 128 x 256
-output tiles.  A CTA that computes more than one tile exercises paths that a
-one-tile-per-CTA launch never reaches: the second accumulator buffer (which
-overlaps the first in TMEM), the drain order of the shared 64-column slots,
-the early hand-back of the accumulator, the ring of TMEM scale regions
-across tile boundaries, and (M > 8192) a last raster group with fewer than
-64 activation tiles.  Each case below runs through the C-ABI and is compared
+The prefill-shaped kernel runs persistent CTA pairs (one pair per two SMs)
+over 256 x 256 output tiles.  A pair that computes more than one tile
+exercises paths that a one-tile-per-pair launch never reaches: the second
+accumulator buffer (which overlaps the first in TMEM), the drain order of
+the shared 64-column slots, the early hand-back of the accumulator to the
+pair's MMA warp, the ring of TMEM scale regions across tile boundaries, and
+(M > 8192) a last raster group with fewer than 32 pair rows (8192
+activation rows).  Each case below runs through the C-ABI and is compared
 element by element with the FP64 oracle: normwise max relative error <= 1e-3
 and relative Frobenius error <= 1e-5 in FP32 output mode, and the BF16
 output is bitwise the BF16 rounding of the FP32 output [picx.dev summary,
@@ -25,10 +26,11 @@ from tests.gpu_helpers import (DEV, assert_gemm_close, check_device_error_word, 
 pytestmark = pytest.mark.gpu
 
 # (M, N, K):
-#   4096 x 4096 x 256  - 32 x 16 = 512 tiles on at most 148 CTAs: 3-4 tiles per CTA
-#   8392 x 512 x 256   - 66 activation tiles: the raster's second group holds 2
-#   2048 x 4103 x 160  - 16 x 17 = 272 tiles, ragged N (odd, so no TMA store
-#                        for f32 rows) and a K tail of half a 64-block
+#   4096 x 4096 x 256  - 16 x 16 = 256 pair tiles on 74 pairs: 3-4 tiles per pair
+#   8392 x 512 x 256   - 33 pair rows: the raster's second group holds 1
+#   2048 x 4103 x 160  - 8 x 17 = 136 pair tiles (about 2 per pair), ragged N
+#                        (odd, so no TMA store for f32 rows) and a K tail of
+#                        half a 64-block
 MULTI_TILE = [(4096, 4096, 256), (8192 + 200, 512, 256), (2048, 4103, 160)]
 
 
